@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 weight-only MoE branch on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode64|decode1|prefill4096|stack30|quantize]
+
+A step is one pass of the whole hot path -- route, permute, gate_up + GELU,
+down, combine -- over one batch of synthetic tokens (the default workload:
+one MoE layer of the Gemma-4-26B-A4B shapes, T=64 decode tokens).  Inputs are
+resident in HBM before the timed region; L2 is flushed (256 MiB write)
+between timed steps, outside the timed events.  Each rank runs its own replica
+(the branch is per-token independent; no collective on the data path);
+`value` is the tokens all ranks processed / max-over-ranks time.
+
+--impl reference times the CPU oracle (numpy, fp64) on a bounded sample of
+the same workload on the host cores; with N>1 only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; decode HBM GB/s vs ~8 TB/s; prefill TFLOP/s vs bf16 peak"
+GU_EXPERT_BYTES = 1408 * 1408 + 1408 * 176 + 4        # packed + scales + global
+DN_EXPERT_BYTES = 2816 * 352 + 2816 * 44 + 4
+EXPERT_BYTES = GU_EXPERT_BYTES + DN_EXPERT_BYTES        # 3,345,416
+ROUTER_BYTES = 128 * 2816 * 2 + 2816 * 2 + 128 * 2       # 726,784 (bf16 proj, scale, pes)
+FLUSH_BYTES = 256 << 20
+
+WORKLOADS = {
+    "decode64": {"T": 64, "layers": 1, "zipf": False,
+                 "desc": "one MoE layer (H=2816, E=128, top-8, I=704, NVFP4 experts), decode T=64"},
+    "decode1": {"T": 1, "layers": 1, "zipf": False, "desc": "one MoE layer, decode T=1"},
+    "prefill4096": {"T": 4096, "layers": 1, "zipf": True,
+                    "desc": "one MoE layer, prefill T=4096, Zipf(1.1)-skewed router bias"},
+    "stack30": {"T": 8, "layers": 30, "zipf": False,
+                "desc": "30 independently seeded MoE layers chained x+=moe(rmsnorm(x)), T=8"},
+    "quantize": {"T": 0, "layers": 0, "zipf": False,
+                 "desc": "nvfp4_quantize of bf16 [128,1408,2816] N(0,0.02) with 0.5% x20 outliers"},
+}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            p = [c.strip() for c in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+# --------------------------------------------------------------- oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+class OracleSample:
+    """The oracle on a bounded sample of the workload: inputs are generated
+    once; each run() times one oracle pass over the sample."""
+
+    def __init__(self, workload: str, wl: dict, tokens: int):
+        import moe_inputs as gen
+        self.workload, self.tokens = workload, tokens
+        if workload == "quantize":
+            self.w = gen.make_quant_weights(4, 1, 1408, 2816)
+            self.what = "oracle quantize of 1 of the 128 expert tensors [1408,2816]"
+            return
+        self.ex = gen.make_experts(0 if wl["layers"] == 1 else 100)
+        self.rt = gen.make_router(1, bias=gen.zipf_bias(7) if wl["zipf"] else None)
+        self.x = gen.make_x(10_000, max(wl["T"], tokens))[:tokens]
+        self.what = f"oracle fp64 forward of {tokens} of the workload's tokens through one layer"
+
+    def run(self):
+        """Returns (value, unit, seconds)."""
+        from oracle import moe as M
+        from oracle import quantize as Q
+        t0 = time.perf_counter()
+        if self.workload == "quantize":
+            Q.quantize(self.w)
+            dt = time.perf_counter() - t0
+            nbytes = self.w.nbytes + self.w.nbytes // 4 + self.w.nbytes // 16 + 4
+            return nbytes / dt / 1e9, "GB/s", dt
+        M.forward(self.x, self.ex, self.rt)
+        dt = time.perf_counter() - t0
+        return self.tokens / dt, "tokens/s", dt
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    tokens = 2 if args.workload != "prefill4096" else 4
+    sample = OracleSample(args.workload, wl, tokens)
+    what = sample.what
+    for _ in range(min(args.warmup, 1)):
+        sample.run()
+    vals, secs = [], []
+    for _ in range(args.steps):
+        v, unit, dt = sample.run()
+        vals.append(v)
+        secs.append(dt)
+    total = sum(secs)
+    value = (tokens * args.steps / total) if unit == "tokens/s" else statistics.mean(vals)
+    if args.workload == "stack30":
+        value /= 30.0   # a stack step runs 30 layers
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "desc": wl["desc"]},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+                         "sample": what + f", {args.steps} steps"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- ours
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import moe_inputs as gen
+    import nvfp4_weight_only_router_b200 as lib
+    from nvfp4_weight_only_router_b200 import build as bld
+
+    if rank == 0 or world == 1:
+        bld.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, tc_peak_sus, peak_kind = measured_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    T = wl["T"]
+    n_pool = 64
+    extra = {}
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    ev_ptrs = None
+
+    if args.workload == "quantize":
+        w = gen.make_quant_weights(4, 128, 1408, 2816)
+        wd = bf(w).to(dev)
+        del w
+        q = torch.empty((128, 1408, 1408), dtype=torch.uint8, device=dev)
+        s = torch.empty((128, 1408, 176), dtype=torch.uint8, device=dev)
+        g = torch.empty((128,), dtype=torch.float32, device=dev)
+        ws = torch.empty(512, dtype=torch.uint8, device=dev)
+        from nvfp4_weight_only_router_b200 import capi
+
+        def step(i):
+            capi.check(capi.nvfp4_quantize(wd.data_ptr(), 128, 1408, 2816, q.data_ptr(), s.data_ptr(),
+                                           g.data_ptr(), ws.data_ptr(), 512,
+                                           torch.cuda.current_stream().cuda_stream))
+        algo_bytes = wd.numel() * 2 + q.numel() + s.numel() + 128 * 4
+        kernels_per_step = 2
+    else:
+        layers = []
+        seeds = [0] if wl["layers"] == 1 else gen.layer_seed_plan(wl["layers"])
+        for li, sd in enumerate(seeds):
+            ex = gen.make_experts(sd)
+            rt = gen.make_router(1 if wl["layers"] == 1 else 1000 + sd,
+                                 bias=gen.zipf_bias(7) if wl["zipf"] else None)
+            layers.append(lib.MoeLayer(lib.Experts.from_host(ex, dev), lib.Router.from_host(rt, dev),
+                                       max_tokens=T))
+            del ex
+        xs_host = np.stack([gen.make_x(10_000 + rank * n_pool + i, T) for i in range(n_pool)])
+        x_pool = bf(xs_host).to(dev)
+        x_pin = bf(xs_host).pin_memory()
+        xs = torch.empty((T, 2816), dtype=torch.bfloat16, device=dev)
+        y = torch.empty_like(xs)
+        y_pin = torch.empty((T, 2816), dtype=torch.bfloat16).pin_memory()
+        res = torch.empty((T, 2816), dtype=torch.float32, device=dev)
+        xn = torch.empty_like(xs)
+
+        def fwd_layer(layer, xin, yout, profiled):
+            from nvfp4_weight_only_router_b200 import capi
+            import ctypes
+            st = torch.cuda.current_stream().cuda_stream
+            if profiled:
+                arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+                capi.check(capi.moe_nvfp4_forward_profiled(
+                    xin.data_ptr(), T, ctypes.byref(layer._xs), ctypes.byref(layer._rs), yout.data_ptr(),
+                    layer.workspace.data_ptr(), layer.workspace.numel(), st, arr))
+            else:
+                layer.forward_into(xin, yout)
+
+        def step_body(profiled):
+            if len(layers) == 1:
+                fwd_layer(layers[0], xs, y, profiled)
+            else:
+                res.copy_(xs.float())
+                lib.residual_rmsnorm(res, None, xn)
+                for li, layer in enumerate(layers):
+                    fwd_layer(layer, xn, y, profiled and li == 0)
+                    lib.residual_rmsnorm(res, y, xn)
+
+        for e in events:   # events must have been recorded once before capture use
+            e.record()
+        torch.cuda.synchronize()
+        # capture one step into a CUDA graph (fixed pointers; inputs rotate into xs)
+        xs.copy_(x_pool[0])
+        step_body(True)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step_body(True)
+        torch.cuda.synchronize()
+
+        def step(i):
+            graph.replay()
+
+        def prepare(i):
+            xs.copy_(x_pool[i % n_pool])
+
+        # route, permute, gate_up, down, combine per layer (+ the chain's rmsnorm kernels)
+        kernels_per_step = 5 * len(layers) + (len(layers) + 1 if len(layers) > 1 else 0)
+
+    # -------- warm-up (at least W steps and at least 1 s, so the clock sampler sees load)
+    sampler = ClockSampler(physical_gpu_index(local_rank))
+    t_end = time.perf_counter() + 1.0
+    i = 0
+    while i < args.warmup or time.perf_counter() < t_end:
+        if args.workload != "quantize":
+            prepare(i)
+        step(i)
+        i += 1
+    torch.cuda.synchronize()
+
+    # -------- timed steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ms, phase_ms, act_counts = [], [], []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        if args.workload != "quantize":
+            prepare(k)
+        start.record()
+        step(k)
+        end.record()
+        torch.cuda.synchronize()
+        step_ms.append(start.elapsed_time(end))
+        if args.workload != "quantize":
+            phase_ms.append([events[j].elapsed_time(events[j + 1]) for j in range(5)])
+            act_counts.append(int((layers[0].views(T)["counts"] > 0).sum().item()))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    # -------- e2e through the public API with host buffers
+    e2e = None
+    if args.workload != "quantize":
+        e_ms = []
+        for k in range(args.steps):
+            flush.zero_()
+            torch.cuda.synchronize()
+            start.record()
+            xs.copy_(x_pin[k % n_pool], non_blocking=True)
+            step_body(False)
+            y_pin.copy_(y, non_blocking=True)
+            end.record()
+            end.synchronize()
+            e_ms.append(start.elapsed_time(end))
+        e_tot = sum(e_ms)
+        if world > 1:
+            t = torch.tensor([e_tot], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_tot = float(t.item())
+        e2e = {"value": world * T * args.steps / (e_tot / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": T * 2816 * 2, "d2h_bytes_per_step": T * 2816 * 2}
+
+    # -------- roofline of the dominant kernel
+    if args.workload == "quantize":
+        value = world * algo_bytes * args.steps / (total_ms / 1e3) / 1e9
+        unit = "GB/s"
+        roof = {"bound": "hbm", "kernel": "nvfp4_quantize (amax + encode)",
+                "achieved": algo_bytes / (ms_per_step / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                "traffic": None, "peak_kind": peak_kind}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        dtype = "u8"
+        e2e = {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+               "note": "weights resident; no host copies in a quantise step"}
+    else:
+        value = world * T * args.steps / (total_ms / 1e3)
+        unit = "tokens/s"
+        ph = np.array(phase_ms)  # [steps, 5]: route, permute, gate_up, down, combine
+        n_act = np.array(act_counts, np.float64)
+        S = T * 8
+        gu_bytes = n_act * GU_EXPERT_BYTES + T * 2816 * 2 + S * 704 * 2
+        gu_flops = 2.0 * S * 1408 * 2816
+        gu_ms = ph[:, 2]
+        if T >= 1024:
+            ach = gu_flops / (gu_ms.mean() / 1e3) / 1e12
+            roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM + GELU", "achieved": ach,
+                    "peak": tc_peak_sus, "unit": "TFLOP/s", "traffic": None, "peak_kind": peak_kind + " sustained",
+                    "algorithmic_per_launch": gu_flops}
+        else:
+            ach = gu_bytes.sum() / (gu_ms.sum() / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": "gate_up grouped GEMV + GELU", "achieved": ach,
+                    "peak": hbm_peak, "unit": "GB/s", "traffic": None, "peak_kind": peak_kind,
+                    "algorithmic_per_launch": float(gu_bytes.mean())}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        step_bytes = n_act * EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2
+        extra = {
+            "phase_ms_mean": dict(zip(["route", "permute", "gate_up", "down", "combine"],
+                                      [float(v) for v in ph.mean(0)])),
+            "active_experts_mean": float(n_act.mean()),
+            # whole-step algorithmic bytes (active experts + router + x + y) per second
+            "step_hbm_gbs": float(step_bytes.mean() * wl["layers"] / (ms_per_step / 1e3) / 1e9),
+            "layer_tflops": float(2.0 * S * (1408 * 2816 + 2816 * 704) * wl["layers"] / (ms_per_step / 1e3) / 1e12),
+        }
+        dtype = "f16xe2m1"
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        tokens = 2 if args.workload != "prefill4096" else 4
+        sample = OracleSample(args.workload, wl, tokens)
+        v, u, dt = sample.run()
+        what = sample.what
+        if args.workload == "stack30":
+            v /= 30.0
+            what += " (value per 30-layer step)"
+        cpu = {"value": v, "unit": u, "cores": blas_threads(), "kind": "oracle",
+               "sample": what + f" ({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+            "config": {"workload": args.workload, "desc": wl["desc"], "T": T,
+                       "l2": "256 MiB flush write between timed steps",
+                       "graph": args.workload != "quantize", "parallelism": f"replicas x{world}"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": kernels_per_step * args.steps, "clocks": clocks,
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    if args.workload != "quantize":
+        del graph
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode64", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

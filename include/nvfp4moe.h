@@ -1,0 +1,217 @@
+/*
+ * nvfp4moe.h -- C ABI of the NVFP4 weight-only (W4A16) sparse MoE branch for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The branch is the sparse half of a Gemma-4-26B-A4B decoder layer
+ * ("Gemma 4 26B-A4B (MoE) - Core AI" card, "Architecture": hidden 2816,
+ * 128 experts, top-8, moe_intermediate 704; the layer dataflow listing and the
+ * router description under it).  Expert weights are NVFP4 ("gemma-4-26B-A4B .
+ * NVFP4A16" release card, "Quantization details"; "Gemma-4-26B-A4B-NVFP4-mlx",
+ * "Quantization recipe"): E2M1 codes packed two per byte, one E4M3 block scale
+ * per 16 consecutive elements along K, one FP32 global scale per expert
+ * projection; w = e2m1 * e4m3 * fp32.  Activations are bf16.
+ *
+ * Conventions for every entry point
+ *   - Pointers named *_dev are device pointers; the caller owns all memory.
+ *     The library never allocates device memory; calls that need scratch
+ *     take a caller-allocated workspace whose size a *_workspace_bytes query
+ *     returns (for the same arguments).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Every call is asynchronous on that stream; none synchronises
+ *     except nvfp4_get_device_status.
+ *   - Arguments are validated on the host before anything is enqueued; an
+ *     invalid call returns an error status and enqueues nothing.
+ *   - Every device pointer must be 16-byte aligned (NVFP4_ERR_ALIGNMENT
+ *     otherwise) and workspaces 256-byte aligned.
+ *   - Errors are returned, never thrown or printed.  A CUDA launch error is
+ *     reported as NVFP4_ERR_CUDA; details via cudaGetLastError.
+ *   - Calls that share a workspace must not overlap on the GPU.
+ *
+ * Tensor layouts (row-major, innermost last)
+ *   x            bf16 [T, H]
+ *   y            bf16 [T, H]
+ *   router.proj  bf16 [E, H]     router.scale bf16 [H]
+ *   router.per_expert_scale bf16 [E]      router.logit_bias f32 [E] or NULL
+ *   gate_up_q    u8   [E, 2I, H/2]   rows 0..I-1 = gate, I..2I-1 = up
+ *   gate_up_s    u8   [E, 2I, H/16]  E4M3 block scales
+ *   gate_up_g    f32  [E]
+ *   down_q       u8   [E, H, I/2]
+ *   down_s       u8   [E, H, I/16]
+ *   down_g       f32  [E]
+ * Byte j of a packed row holds element 2j in its low nibble and element 2j+1
+ * in its high nibble.  The sign bit of an E2M1 code is bit 3.
+ */
+#ifndef NVFP4MOE_H
+#define NVFP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NVFP4MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define NVFP4MOE_API __attribute__((visibility("default")))
+#else
+#define NVFP4MOE_API
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,   /* null pointer, non-positive or inconsistent size */
+  NVFP4_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+  NVFP4_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the query returned */
+  NVFP4_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  NVFP4_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (device status) */
+  NVFP4_ERR_UNSUPPORTED = 6,   /* valid but not implemented shape (see each call) */
+  NVFP4_ERR_DEVICE = 7         /* a kernel detected bad input data (device status) */
+} nvfp4_status;
+
+/* Router parameters ("Gemma 4 26B-A4B (MoE) - Core AI", router description
+ * under the layer dataflow listing).  All pointers are device pointers. */
+typedef struct {
+  const void* proj;              /* bf16 [E, H] */
+  const void* scale;             /* bf16 [H] */
+  const void* per_expert_scale;  /* bf16 [E] */
+  const float* logit_bias;       /* f32 [E], added to the logits; NULL = none */
+  int32_t E;                     /* number of experts: must be 128 */
+  int32_t H;                     /* hidden size: multiple of 128, <= 16384 */
+  int32_t top_k;                 /* must be 8 */
+  float eps;                     /* RMSNorm epsilon (the pages are silent; 1e-6) */
+} moe_router;
+
+/* NVFP4 expert stacks.  All pointers are device pointers. */
+typedef struct {
+  const uint8_t* gate_up_q;  /* [E, 2I, H/2] */
+  const uint8_t* gate_up_s;  /* [E, 2I, H/16] */
+  const float* gate_up_g;    /* [E] */
+  const uint8_t* down_q;     /* [E, H, I/2] */
+  const uint8_t* down_s;     /* [E, H, I/16] */
+  const float* down_g;       /* [E] */
+  int32_t E;                 /* must be 128 */
+  int32_t H;                 /* must be 2816 */
+  int32_t I;                 /* must be 704 */
+} moe_experts;
+
+/* ---------------------------------------------------------------------------
+ * nvfp4_quantize: bf16 weights -> NVFP4.
+ * Source: "Gemma-4-26B-A4B-it-NVFP4" page, block-scale formulas (S_block =
+ * max|w|/6, q = clip(round(w/S), -6, 6)), in the two-level form of the
+ * NVFP4A16 card ("Quantization details").  For each tensor e (one per expert):
+ *   G      = f32(amax_e) / 2688                    (2688 = 6 * 448)
+ *   s_b    = E4M3_rne_satfinite((amax_b / 6) / G)  per block of 16 along K
+ *   d_b    = f32(s_b) * G
+ *   code_i = E2M1_rne(w_i / d_b), saturating at 6, sign bit = sign bit of w_i
+ * each step one correctly rounded fp32 operation; ties go to the even code.
+ * A block with d_b == 0 (all-zero block or tensor) gets scale 0 and codes that
+ * carry only the sign bit.
+ *   w_dev  bf16 [E, N, K] (in)      q_dev u8 [E, N, K/2] (out)
+ *   s_dev  u8 [E, N, K/16] (out)    g_dev f32 [E] (out)
+ * Requires E >= 1, N >= 1, K >= 16, K % 32 == 0, N * K < 2^31.  NaN/Inf
+ * inputs are not supported (their codes are unspecified).
+ * Workspace: nvfp4_quantize_workspace_bytes(E, N, K) bytes, 256-aligned.
+ * ------------------------------------------------------------------------- */
+NVFP4MOE_API size_t nvfp4_quantize_workspace_bytes(int64_t E, int64_t N, int64_t K);
+NVFP4MOE_API nvfp4_status nvfp4_quantize(const void* w_dev, int64_t E, int64_t N, int64_t K,
+                            uint8_t* q_dev, uint8_t* s_dev, float* g_dev,
+                            void* ws_dev, size_t ws_bytes, void* stream);
+
+/* nvfp4_dequantize: w = e2m1 * e4m3 * G rounded once to fp32 ("Gemma-4-26B-A4B-
+ * NVFP4-mlx", "Quantization recipe": E2M1 x per-16 E4M3 x per-tensor F32).
+ * Same layouts and limits as nvfp4_quantize; out_dev f32 [E, N, K].  No
+ * workspace. */
+NVFP4MOE_API nvfp4_status nvfp4_dequantize(const uint8_t* q_dev, const uint8_t* s_dev, const float* g_dev,
+                              int64_t E, int64_t N, int64_t K, float* out_dev, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route: the router ("Gemma 4 26B-A4B (MoE) - Core AI", router
+ * description): r = x / sqrt(mean(x^2) + eps) * scale * H^-0.5;
+ * logits = proj r (+ logit_bias); p = softmax(logits) in fp32 over all E;
+ * the top_k largest p; weights = p_sel / sum(p_sel) * per_expert_scale[ids].
+ * fp32 arithmetic throughout (the x*scale products are carried exactly).
+ *   x_dev    bf16 [T, H] (in)
+ *   ids_dev  int32 [T, top_k] (out), by descending p; the selection compares
+ *            the fp32 logits (softmax is monotone), equal logits -> lower id first
+ *   w_dev    f32 [T, top_k] (out)
+ * Requires 1 <= T <= 65536, E == 128, top_k == 8, H % 128 == 0, H <= 16384.
+ * Workspace: moe_route_workspace_bytes(T, router) bytes.
+ * ------------------------------------------------------------------------- */
+NVFP4MOE_API size_t moe_route_workspace_bytes(int32_t T, const moe_router* router);
+NVFP4MOE_API nvfp4_status moe_route(const void* x_dev, int32_t T, const moe_router* router,
+                       int32_t* ids_dev, float* w_dev,
+                       void* ws_dev, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_nvfp4_forward: y = sum_j w_j * expert_{id_j}(x) for every token
+ * ("Gemma 4 26B-A4B (MoE) - Core AI", layer dataflow listing: the experts'
+ * outputs combined as sum_k w_k h2_k; experts GELU-tanh gated).  Both the
+ * router and the experts read x.  Per expert e and routed token x:
+ *   gate = G_gu[e] * (Wq_gate[e] x),  up = G_gu[e] * (Wq_up[e] x)
+ *   h    = gelu_tanh(gate) * up
+ *   out  = G_d[e] * (Wq_down[e] h)
+ * where Wq = e2m1 * e4m3 is exact in f16.  x and h enter the tensor cores as
+ * f16 (x converted with saturation to +-65504; h rounded to f16), products are
+ * accumulated in fp32, the combine is fp32, y is rounded once to bf16.
+ *   x_dev bf16 [T, H] (in), y_dev bf16 [T, H] (out)
+ * Requires 1 <= T <= 65536, E == 128, H == 2816, I == 704, top_k == 8.
+ * Workspace: moe_forward_workspace_bytes(T, experts, router) bytes.
+ * ------------------------------------------------------------------------- */
+NVFP4MOE_API size_t moe_forward_workspace_bytes(int32_t T, const moe_experts* experts, const moe_router* router);
+NVFP4MOE_API nvfp4_status moe_nvfp4_forward(const void* x_dev, int32_t T, const moe_experts* experts,
+                               const moe_router* router, void* y_dev,
+                               void* ws_dev, size_t ws_bytes, void* stream);
+
+/* moe_nvfp4_forward_profiled: moe_nvfp4_forward that also records CUDA
+ * events between its phases on `stream`.  phase_events points to 6 cudaEvent_t
+ * (passed as void*; a NULL entry is skipped): [0] before the first kernel,
+ * [1] after the router, [2] after the permutation, [3] after gate_up + GELU,
+ * [4] after down, [5] after the combine.  Results are identical to
+ * moe_nvfp4_forward. */
+NVFP4MOE_API nvfp4_status moe_nvfp4_forward_profiled(const void* x_dev, int32_t T,
+                                                     const moe_experts* experts,
+                                                     const moe_router* router, void* y_dev,
+                                                     void* ws_dev, size_t ws_bytes, void* stream,
+                                                     void* const* phase_events);
+
+/* Byte offsets, inside a forward workspace, of the intermediate results a
+ * finished moe_nvfp4_forward leaves behind (for inspection and tests):
+ *   ids int32 [T, 8], weights f32 [T, 8] (the router's outputs),
+ *   counts int32 [E], offsets int32 [E+1] (exclusive prefix of counts),
+ *   sorted_slot int32 [T*8] (slots t*8+j grouped by expert, stable),
+ *   slot_pos int32 [T*8] (inverse permutation),
+ *   h f16 [T*8, I] (gated hidden, rows in sorted_slot order). */
+typedef struct {
+  size_t ids, weights, counts, offsets, sorted_slot, slot_pos, h;
+} moe_forward_views;
+NVFP4MOE_API nvfp4_status moe_forward_workspace_views(int32_t T, const moe_experts* experts,
+                                         const moe_router* router, moe_forward_views* out);
+
+/* ---------------------------------------------------------------------------
+ * moe_residual_rmsnorm: one link of a chained layer stack,
+ *   res += y (if y_dev != NULL);  x_out = bf16(res / sqrt(mean(res^2) + eps))
+ * (scale-free RMSNorm as in the router description).  Used to chain layers as
+ * x_{l+1} = x_l + moe_l(rmsnorm(x_l)) with an fp32 residual.
+ *   res_dev f32 [T, H] (in/out), y_dev bf16 [T, H] or NULL, x_out_dev bf16 [T, H]
+ * Requires 1 <= T <= 65536, H % 8 == 0, H <= 16384.  No workspace.
+ * ------------------------------------------------------------------------- */
+NVFP4MOE_API nvfp4_status moe_residual_rmsnorm(float* res_dev, const void* y_dev, void* x_out_dev,
+                                  int32_t T, int32_t H, float eps, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Device status: kernels record data errors (an expert id out of range) and
+ * bounded waits that gave up in a per-device status word instead of faulting.
+ * nvfp4_get_device_status synchronises `stream`, returns the first recorded
+ * error (NVFP4_OK if none) and clears the word.
+ * ------------------------------------------------------------------------- */
+NVFP4MOE_API nvfp4_status nvfp4_get_device_status(void* stream);
+
+NVFP4MOE_API const char* nvfp4_status_string(nvfp4_status status);
+NVFP4MOE_API int nvfp4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4MOE_H */

@@ -1,0 +1,196 @@
+"""torch conveniences over the C ABI: allocate outputs and workspaces with
+torch (device memory plumbing) and pass their pointers to the library calls
+on torch's current CUDA stream."""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+
+import torch
+
+from . import capi
+from .capi import check
+
+E, H, I, TOP_K = 128, 2816, 704, 8
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+@dataclasses.dataclass
+class Router:
+    """Router parameters on the device: proj bf16 [E, H], scale bf16 [H],
+    per_expert_scale bf16 [E], optional logit_bias f32 [E]."""
+    proj: torch.Tensor
+    scale: torch.Tensor
+    per_expert_scale: torch.Tensor
+    logit_bias: torch.Tensor | None = None
+    eps: float = 1e-6
+    top_k: int = TOP_K
+
+    def c_struct(self) -> capi.moe_router:
+        return capi.moe_router(_ptr(self.proj), _ptr(self.scale), _ptr(self.per_expert_scale),
+                               _ptr(self.logit_bias), self.proj.shape[0], self.proj.shape[1],
+                               self.top_k, self.eps)
+
+    @staticmethod
+    def from_host(r, device="cuda") -> "Router":
+        """From a host router of bf16 bit patterns (numpy uint16 arrays)."""
+        def bf(a):
+            return torch.from_numpy(a.view("int16")).view(torch.bfloat16).to(device)
+        bias = None if r.logit_bias is None else torch.from_numpy(r.logit_bias).to(device)
+        return Router(bf(r.proj), bf(r.scale), bf(r.per_expert_scale), bias, float(r.eps), int(r.top_k))
+
+
+@dataclasses.dataclass
+class Experts:
+    """NVFP4 expert stacks on the device (layouts of include/nvfp4moe.h)."""
+    gate_up_q: torch.Tensor
+    gate_up_s: torch.Tensor
+    gate_up_g: torch.Tensor
+    down_q: torch.Tensor
+    down_s: torch.Tensor
+    down_g: torch.Tensor
+
+    def c_struct(self) -> capi.moe_experts:
+        return capi.moe_experts(_ptr(self.gate_up_q), _ptr(self.gate_up_s), _ptr(self.gate_up_g),
+                                _ptr(self.down_q), _ptr(self.down_s), _ptr(self.down_g),
+                                self.gate_up_q.shape[0], self.gate_up_q.shape[2] * 2,
+                                self.down_q.shape[2] * 2)
+
+    @staticmethod
+    def from_host(x, device="cuda") -> "Experts":
+        t = lambda a: torch.from_numpy(a).to(device)  # noqa: E731
+        return Experts(t(x.gate_up_q), t(x.gate_up_s), t(x.gate_up_g), t(x.down_q), t(x.down_s),
+                       t(x.down_g))
+
+    def nbytes_per_expert(self) -> int:
+        return sum(a[0].numel() * a.element_size() for a in
+                   (self.gate_up_q, self.gate_up_s, self.down_q, self.down_s)) + 8
+
+
+# ------------------------------------------------------------------ quantise
+def quantize(w: torch.Tensor, stream=None):
+    """bf16 [E, N, K] -> (q uint8 [E, N, K/2], s uint8 [E, N, K/16], g f32 [E])."""
+    if w.dtype != torch.bfloat16 or w.dim() != 3:
+        raise ValueError("w must be a bf16 tensor [E, N, K]")
+    Ee, N, K = w.shape
+    dev = w.device
+    q = torch.empty((Ee, N, K // 2), dtype=torch.uint8, device=dev)
+    s = torch.empty((Ee, N, K // 16), dtype=torch.uint8, device=dev)
+    g = torch.empty((Ee,), dtype=torch.float32, device=dev)
+    nbytes = capi.nvfp4_quantize_workspace_bytes(Ee, N, K)
+    ws = _workspace(nbytes, dev)
+    check(capi.nvfp4_quantize(_ptr(w), Ee, N, K, _ptr(q), _ptr(s), _ptr(g), _ptr(ws), ws.numel(),
+                              _stream(stream)), "nvfp4_quantize")
+    return q, s, g
+
+
+def dequantize(q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, stream=None) -> torch.Tensor:
+    Ee, N, K2 = q.shape
+    out = torch.empty((Ee, N, K2 * 2), dtype=torch.float32, device=q.device)
+    check(capi.nvfp4_dequantize(_ptr(q), _ptr(s), _ptr(g), Ee, N, K2 * 2, _ptr(out), _stream(stream)),
+          "nvfp4_dequantize")
+    return out
+
+
+# --------------------------------------------------------------------- route
+def route(x: torch.Tensor, router: Router, stream=None):
+    """bf16 [T, H] -> (ids int32 [T, 8], weights f32 [T, 8])."""
+    T = x.shape[0]
+    rs = router.c_struct()
+    ids = torch.empty((T, router.top_k), dtype=torch.int32, device=x.device)
+    w = torch.empty((T, router.top_k), dtype=torch.float32, device=x.device)
+    nbytes = capi.moe_route_workspace_bytes(T, ctypes.byref(rs))
+    ws = _workspace(nbytes, x.device)
+    check(capi.moe_route(_ptr(x), T, ctypes.byref(rs), _ptr(ids), _ptr(w), _ptr(ws), ws.numel(),
+                         _stream(stream)), "moe_route")
+    return ids, w
+
+
+# ------------------------------------------------------------------- forward
+class MoeLayer:
+    """One NVFP4 MoE branch: holds the device parameters and a workspace sized
+    for up to `max_tokens` tokens.  Calls of one layer must not overlap on the
+    GPU (they share the workspace)."""
+
+    def __init__(self, experts: Experts, router: Router, max_tokens: int):
+        self.experts, self.router = experts, router
+        self._xs, self._rs = experts.c_struct(), router.c_struct()
+        self.max_tokens = int(max_tokens)
+        nbytes = capi.moe_forward_workspace_bytes(self.max_tokens, ctypes.byref(self._xs),
+                                                  ctypes.byref(self._rs))
+        if nbytes == 0:
+            raise ValueError("unsupported experts/router configuration")
+        self.workspace = _workspace(nbytes, experts.gate_up_q.device)
+
+    def workspace_bytes(self, T: int) -> int:
+        return capi.moe_forward_workspace_bytes(T, ctypes.byref(self._xs), ctypes.byref(self._rs))
+
+    def forward_into(self, x: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"T={T} exceeds max_tokens={self.max_tokens}")
+        check(capi.moe_nvfp4_forward(_ptr(x), T, ctypes.byref(self._xs), ctypes.byref(self._rs),
+                                     _ptr(y), _ptr(self.workspace), self.workspace.numel(),
+                                     _stream(stream)), "moe_nvfp4_forward")
+        return y
+
+    def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        y = torch.empty_like(x)
+        return self.forward_into(x, y, stream)
+
+    def views(self, T: int) -> dict:
+        """Intermediate results of the last forward of T tokens, as torch views
+        of the workspace (see moe_forward_views in the header)."""
+        return forward_views(self, T)
+
+
+def forward_views(layer: MoeLayer, T: int) -> dict:
+    v = capi.moe_forward_views()
+    check(capi.moe_forward_workspace_views(T, ctypes.byref(layer._xs), ctypes.byref(layer._rs),
+                                           ctypes.byref(v)), "moe_forward_workspace_views")
+    ws = layer.workspace
+    S = T * TOP_K
+
+    def view(off, n, dtype):
+        item = torch.empty((), dtype=dtype).element_size()
+        return ws[off:off + n * item].view(dtype)
+
+    return {
+        "ids": view(v.ids, S, torch.int32).view(T, TOP_K),
+        "weights": view(v.weights, S, torch.float32).view(T, TOP_K),
+        "counts": view(v.counts, E, torch.int32),
+        "offsets": view(v.offsets, E + 1, torch.int32),
+        "sorted_slot": view(v.sorted_slot, S, torch.int32),
+        "slot_pos": view(v.slot_pos, S, torch.int32),
+        "h": view(v.h, S * I, torch.float16).view(S, I),
+    }
+
+
+def residual_rmsnorm(res: torch.Tensor, y: torch.Tensor | None, x_out: torch.Tensor, eps: float = 1e-6,
+                     stream=None) -> None:
+    T, Hh = res.shape
+    check(capi.moe_residual_rmsnorm(_ptr(res), _ptr(y), _ptr(x_out), T, Hh, eps, _stream(stream)),
+          "moe_residual_rmsnorm")
+
+
+def device_status(stream=None) -> int:
+    return capi.nvfp4_get_device_status(_stream(stream))

@@ -1,0 +1,376 @@
+// C ABI of the NVFP4 MoE library: argument validation, workspace layout and
+// launch sequencing on the caller's stream.  See include/nvfp4moe.h.
+#include <cmath>
+#include <mutex>
+
+#include "../../include/nvfp4moe.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace nvfp4moe;
+
+namespace {
+
+// Per-device status word (see nvfp4_get_device_status).
+__device__ int g_device_status;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+int* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// ------------------------------------------------------------------ layouts
+struct Region {
+  size_t off = 0, bytes = 0;
+};
+
+struct Alloc {
+  size_t cur = 0;
+  Region take(size_t bytes) {
+    Region r;
+    r.off = cur;
+    r.bytes = bytes;
+    cur = round_up(cur + bytes, 256);
+    return r;
+  }
+};
+
+struct RouteLayout {
+  int ntiles = 0, ksplit = 0, segs_per_split = 0;
+  Region counters, part_logits, part_ss;
+};
+
+RouteLayout route_layout(Alloc& al, int T, int H) {
+  RouteLayout L;
+  L.ntiles = (T + 15) / 16;
+  const int nseg = H / kSegK;
+  if (T <= 256) {
+    L.ksplit = nseg;
+    L.segs_per_split = 1;
+  } else {
+    L.ksplit = 1;
+    L.segs_per_split = nseg;
+  }
+  L.counters = al.take(sizeof(int) * L.ntiles);
+  L.part_logits = al.take(sizeof(float) * (size_t)L.ksplit * T * kE);
+  L.part_ss = al.take(sizeof(float) * (size_t)L.ksplit * T);
+  return L;
+}
+
+struct FwdLayout {
+  Region meta;
+  RouteLayout route;
+  Region ids, wts, chunk_count, chunk_base, local_rank, sorted, pos, x16, h, obuf, yacc;
+  int S = 0, nchunks = 0, mode = 0;
+  size_t total = 0;
+};
+
+constexpr int kDeterministicMaxT = 256;  // per-slot combine buffer up to this T
+
+FwdLayout fwd_layout(int T) {
+  FwdLayout L;
+  Alloc al;
+  L.S = T * kTopK;
+  L.nchunks = (L.S + 1023) / 1024;
+  L.mode = (T <= kDeterministicMaxT) ? 0 : 1;
+  // zeroed on entry: meta (includes the permute counter) and the router counters
+  L.meta = al.take(sizeof(int) * kMetaInts);
+  L.route = route_layout(al, T, kH);
+  L.ids = al.take(sizeof(int) * L.S);
+  L.wts = al.take(sizeof(float) * L.S);
+  L.chunk_count = al.take(sizeof(int) * (size_t)L.nchunks * kE);
+  L.chunk_base = al.take(sizeof(int) * (size_t)L.nchunks * kE);
+  L.local_rank = al.take(sizeof(int) * L.S);
+  L.sorted = al.take(sizeof(int) * L.S);
+  L.pos = al.take(sizeof(int) * L.S);
+  L.x16 = al.take(sizeof(__half) * (size_t)T * kH);
+  L.h = al.take(sizeof(__half) * (size_t)L.S * kI);
+  if (L.mode == 0)
+    L.obuf = al.take(sizeof(float) * (size_t)L.S * kH);
+  else
+    L.yacc = al.take(sizeof(float) * (size_t)T * kH);
+  L.total = al.cur;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, const Region& r) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + r.off);
+}
+
+nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+nvfp4_status check_router(const moe_router* r, bool forward) {
+  if (!r || !r->proj || !r->scale || !r->per_expert_scale) return NVFP4_ERR_INVALID_ARG;
+  if (r->E <= 0 || r->H <= 0 || r->top_k <= 0 || !(r->eps >= 0.f) || !std::isfinite(r->eps))
+    return NVFP4_ERR_INVALID_ARG;
+  if (r->E != kE || r->top_k != kTopK) return NVFP4_ERR_UNSUPPORTED;
+  if (forward ? (r->H != kH) : (r->H % kSegK != 0 || r->H > 16384)) return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned(r->proj, 16) || !aligned(r->scale, 16) || !aligned(r->per_expert_scale, 16) ||
+      (r->logit_bias && !aligned(r->logit_bias, 16)))
+    return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+nvfp4_status check_experts(const moe_experts* x) {
+  if (!x || !x->gate_up_q || !x->gate_up_s || !x->gate_up_g || !x->down_q || !x->down_s ||
+      !x->down_g)
+    return NVFP4_ERR_INVALID_ARG;
+  if (x->E <= 0 || x->H <= 0 || x->I <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (x->E != kE || x->H != kH || x->I != kI) return NVFP4_ERR_UNSUPPORTED;
+  const void* ps[] = {x->gate_up_q, x->gate_up_s, x->gate_up_g, x->down_q, x->down_s, x->down_g};
+  for (const void* p : ps)
+    if (!aligned(p, 16)) return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+RouteArgs make_route_args(const void* x, int T, const moe_router* r, const RouteLayout& L, void* ws,
+                          int32_t* ids, float* wts, __half* x16, int* status) {
+  RouteArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.proj = static_cast<const uint16_t*>(r->proj);
+  a.scale = static_cast<const uint16_t*>(r->scale);
+  a.pes = static_cast<const uint16_t*>(r->per_expert_scale);
+  a.bias = r->logit_bias;
+  a.T = T;
+  a.H = r->H;
+  a.ksplit = L.ksplit;
+  a.segs_per_split = L.segs_per_split;
+  a.eps = r->eps;
+  a.inv_sqrt_h = (float)(1.0 / std::sqrt((double)r->H));
+  a.part_logits = at<float>(ws, L.part_logits);
+  a.part_ss = at<float>(ws, L.part_ss);
+  a.tile_counter = at<int>(ws, L.counters);
+  a.ids = ids;
+  a.wts = wts;
+  a.x16 = x16;
+  a.status = status;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_abi_version(void) { return NVFP4MOE_ABI_VERSION; }
+
+const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_ALIGNMENT: return "misaligned pointer";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported shape";
+    case NVFP4_ERR_DEVICE: return "invalid data detected on the device";
+  }
+  return "unknown status";
+}
+
+// ---------------------------------------------------------------- quantize
+static nvfp4_status check_quant_dims(int64_t E, int64_t N, int64_t K) {
+  if (E < 1 || N < 1 || K < 16) return NVFP4_ERR_INVALID_ARG;
+  if (K % 32 != 0) return NVFP4_ERR_UNSUPPORTED;
+  if (N * K >= (int64_t(1) << 31) || E > (int64_t(1) << 20)) return NVFP4_ERR_UNSUPPORTED;
+  return NVFP4_OK;
+}
+
+size_t nvfp4_quantize_workspace_bytes(int64_t E, int64_t N, int64_t K) {
+  if (check_quant_dims(E, N, K) != NVFP4_OK) return 0;
+  return round_up(sizeof(uint32_t) * (size_t)E, 256);
+}
+
+nvfp4_status nvfp4_quantize(const void* w, int64_t E, int64_t N, int64_t K, uint8_t* q, uint8_t* s,
+                            float* g, void* ws, size_t ws_bytes, void* stream) {
+  nvfp4_status st = check_quant_dims(E, N, K);
+  if (st != NVFP4_OK) return st;
+  if (!w || !q || !s || !g) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 16) || !aligned(s, 16) || !aligned(g, 16))
+    return NVFP4_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < nvfp4_quantize_workspace_bytes(E, N, K)) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
+  return cuda_status(launch_quantize(static_cast<const uint16_t*>(w), E, N, K, q, s, g,
+                                     static_cast<uint32_t*>(ws), as_stream(stream)));
+}
+
+nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* s, const float* g, int64_t E,
+                              int64_t N, int64_t K, float* out, void* stream) {
+  nvfp4_status st = check_quant_dims(E, N, K);
+  if (st != NVFP4_OK) return st;
+  if (!q || !s || !g || !out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(s, 16) || !aligned(g, 16) || !aligned(out, 16))
+    return NVFP4_ERR_ALIGNMENT;
+  return cuda_status(launch_dequantize(q, s, g, E, N, K, out, as_stream(stream)));
+}
+
+// ------------------------------------------------------------------- route
+size_t moe_route_workspace_bytes(int32_t T, const moe_router* r) {
+  if (T < 1 || T > 65536 || check_router(r, false) != NVFP4_OK) return 0;
+  Alloc al;
+  route_layout(al, T, r->H);
+  return al.cur;
+}
+
+nvfp4_status moe_route(const void* x, int32_t T, const moe_router* r, int32_t* ids, float* w,
+                       void* ws, size_t ws_bytes, void* stream) {
+  if (T < 1 || T > 65536 || !x || !ids || !w) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_router(r, false);
+  if (st != NVFP4_OK) return st;
+  if (!aligned(x, 16) || !aligned(ids, 16) || !aligned(w, 16)) return NVFP4_ERR_ALIGNMENT;
+  const size_t need = moe_route_workspace_bytes(T, r);
+  if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
+  Alloc al;
+  RouteLayout L = route_layout(al, T, r->H);
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaMemsetAsync(at<int>(ws, L.counters), 0, L.counters.bytes, s);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  RouteArgs a = make_route_args(x, T, r, L, ws, ids, w, nullptr, device_status_ptr());
+  return cuda_status(launch_route(a, s));
+}
+
+// ----------------------------------------------------------------- forward
+size_t moe_forward_workspace_bytes(int32_t T, const moe_experts* ex, const moe_router* r) {
+  if (T < 1 || T > 65536 || check_experts(ex) != NVFP4_OK || check_router(r, true) != NVFP4_OK)
+    return 0;
+  return fwd_layout(T).total;
+}
+
+nvfp4_status moe_forward_workspace_views(int32_t T, const moe_experts* ex, const moe_router* r,
+                                         moe_forward_views* out) {
+  if (!out || T < 1 || T > 65536) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_experts(ex);
+  if (st == NVFP4_OK) st = check_router(r, true);
+  if (st != NVFP4_OK) return st;
+  FwdLayout L = fwd_layout(T);
+  out->ids = L.ids.off;
+  out->weights = L.wts.off;
+  out->counts = L.meta.off + sizeof(int) * kMetaCounts;
+  out->offsets = L.meta.off + sizeof(int) * kMetaOffsets;
+  out->sorted_slot = L.sorted.off;
+  out->slot_pos = L.pos.off;
+  out->h = L.h.off;
+  return NVFP4_OK;
+}
+
+static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex,
+                                 const moe_router* r, void* y, void* ws, size_t ws_bytes,
+                                 void* stream, void* const* ev) {
+  if (T < 1 || T > 65536 || !x || !y) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_experts(ex);
+  if (st == NVFP4_OK) st = check_router(r, true);
+  if (st != NVFP4_OK) return st;
+  if (!aligned(x, 16) || !aligned(y, 16)) return NVFP4_ERR_ALIGNMENT;
+  const FwdLayout L = fwd_layout(T);
+  if (!ws || ws_bytes < L.total) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = as_stream(stream);
+  int* status = device_status_ptr();
+  auto mark = [&](int i) -> bool {
+    return !ev || !ev[i] || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
+  };
+  if (!mark(0)) return NVFP4_ERR_CUDA;
+
+  // meta and router counters are contiguous at the start of the workspace
+  const size_t zero_bytes = L.route.counters.off + L.route.counters.bytes;
+  cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, s);
+  if (e == cudaSuccess && L.mode == 1) e = cudaMemsetAsync(at<float>(ws, L.yacc), 0, L.yacc.bytes, s);
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+
+  int32_t* ids = at<int32_t>(ws, L.ids);
+  float* wts = at<float>(ws, L.wts);
+  __half* x16 = at<__half>(ws, L.x16);
+  RouteArgs ra = make_route_args(x, T, r, L.route, ws, ids, wts, x16, status);
+  if ((e = launch_route(ra, s)) != cudaSuccess || !mark(1)) return NVFP4_ERR_CUDA;
+
+  PermuteArgs pa;
+  pa.ids = ids;
+  pa.S = L.S;
+  pa.nchunks = L.nchunks;
+  pa.meta = at<int>(ws, L.meta);
+  pa.chunk_count = at<int>(ws, L.chunk_count);
+  pa.chunk_base = at<int>(ws, L.chunk_base);
+  pa.local_rank = at<int>(ws, L.local_rank);
+  pa.sorted_slot = at<int>(ws, L.sorted);
+  pa.slot_pos = at<int>(ws, L.pos);
+  pa.status = status;
+  if ((e = launch_permute(pa, s)) != cudaSuccess || !mark(2)) return NVFP4_ERR_CUDA;
+
+  ExpertArgs xa;
+  xa.gu_q = ex->gate_up_q;
+  xa.gu_s = ex->gate_up_s;
+  xa.gu_g = ex->gate_up_g;
+  xa.dn_q = ex->down_q;
+  xa.dn_s = ex->down_s;
+  xa.dn_g = ex->down_g;
+  xa.x16 = x16;
+  xa.meta = pa.meta;
+  xa.sorted_slot = pa.sorted_slot;
+  xa.slot_pos = pa.slot_pos;
+  xa.wts = wts;
+  xa.h = at<__half>(ws, L.h);
+  xa.obuf = L.mode == 0 ? at<float>(ws, L.obuf) : nullptr;
+  xa.yacc = L.mode == 1 ? at<float>(ws, L.yacc) : nullptr;
+  xa.y = y;
+  xa.T = T;
+  xa.max_active = L.S < kE ? L.S : kE;
+  xa.mode = L.mode;
+  xa.status = status;
+  if ((e = launch_gate_up_gemv(xa, s)) != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
+  if ((e = launch_down_gemv(xa, s)) != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
+  if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return NVFP4_ERR_CUDA;
+  return NVFP4_OK;
+}
+
+nvfp4_status moe_nvfp4_forward(const void* x, int32_t T, const moe_experts* ex, const moe_router* r,
+                               void* y, void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, nullptr);
+}
+
+nvfp4_status moe_nvfp4_forward_profiled(const void* x, int32_t T, const moe_experts* ex,
+                                        const moe_router* r, void* y, void* ws, size_t ws_bytes,
+                                        void* stream, void* const* phase_events) {
+  return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, phase_events);
+}
+
+// ------------------------------------------------------------ chain helper
+nvfp4_status moe_residual_rmsnorm(float* res, const void* y, void* x_out, int32_t T, int32_t H,
+                                  float eps, void* stream) {
+  if (!res || !x_out || T < 1 || T > 65536 || H < 8 || H % 8 != 0 || H > 16384 ||
+      !(eps >= 0.f) || !std::isfinite(eps))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(res, 16) || !aligned(x_out, 16) || (y && !aligned(y, 16))) return NVFP4_ERR_ALIGNMENT;
+  return cuda_status(launch_residual_rmsnorm(res, static_cast<const uint16_t*>(y),
+                                             static_cast<uint16_t*>(x_out), T, H, eps,
+                                             as_stream(stream)));
+}
+
+// ----------------------------------------------------------- device status
+nvfp4_status nvfp4_get_device_status(void* stream) {
+  int* p = device_status_ptr();
+  if (!p) return NVFP4_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  int v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (v != 0 && cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  return static_cast<nvfp4_status>(v);
+}
+
+}  // extern "C"

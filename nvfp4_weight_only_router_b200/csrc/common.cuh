@@ -1,0 +1,142 @@
+// Shared device helpers of the NVFP4 MoE library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4moe {
+
+// Layer constants of the Gemma-4-26B-A4B MoE branch ("Gemma 4 26B-A4B (MoE) -
+// Core AI", "Architecture" table).
+constexpr int kH = 2816;          // hidden size
+constexpr int kI = 704;           // moe_intermediate_size
+constexpr int kE = 128;           // routed experts
+constexpr int kTopK = 8;          // experts per token
+constexpr int kBlock = 16;        // elements per E4M3 block scale
+
+// Packed row geometry.
+constexpr int kGuRowBytes = kH / 2;        // 1408: one gate_up row, two codes per byte
+constexpr int kGuScaleRow = kH / kBlock;   // 176
+constexpr int kDnRowBytes = kI / 2;        // 352
+constexpr int kDnScaleRow = kI / kBlock;   // 44
+
+// A "segment" is 128 consecutive K elements = 64 packed bytes: four lanes of a
+// quad each hold one 16-byte chunk (32 elements) of it.
+constexpr int kSegK = 128;
+constexpr int kGuSegs = kH / kSegK;              // 22
+constexpr int kDnSegs = (kI + kSegK - 1) / kSegK; // 6 (the last one half full)
+
+// Device status codes (mirror nvfp4_status).
+constexpr int kStatusTimeout = 5;
+constexpr int kStatusDevice = 7;
+
+// Layout of the small integer "meta" block at the start of a forward
+// workspace.
+constexpr int kMetaCounts = 0;      // [E] tokens routed to each expert
+constexpr int kMetaOffsets = 128;   // [E+1] exclusive prefix of counts
+constexpr int kMetaAct = 260;       // [E] ids of experts with count > 0, ascending
+constexpr int kMetaNAct = 388;      // number of active experts
+constexpr int kMetaPermCounter = 392;  // arrival counter of the permute kernel
+constexpr int kMetaInts = 512;
+
+__device__ __forceinline__ void record_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// ------------------------------------------------------------- conversions
+// Four packed bytes (eight E2M1 codes) -> four f16x2 registers.  Register i
+// holds byte i: its low nibble in the low half, its high nibble in the high
+// half.  The conversion is exact (every E2M1 value is an f16).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&o)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
+// Two E4M3 bytes (low byte first) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t o;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(o) : "h"(v));
+  return o;
+}
+
+// f16x2 multiply (used on exact products only: e2m1 * e4m3 fits in f16).
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  uint32_t o;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(o) : "r"(a), "r"(b));
+  return o;
+}
+
+// Broadcast the low / high half of an f16x2 to both halves.
+__device__ __forceinline__ uint32_t bcast_lo(uint32_t v) { return __byte_perm(v, v, 0x1010); }
+__device__ __forceinline__ uint32_t bcast_hi(uint32_t v) { return __byte_perm(v, v, 0x3232); }
+
+// fp32 -> f16 with saturation to +-65504 (finite inputs).
+__device__ __forceinline__ __half f32_to_f16_sat(float v) {
+  v = fminf(fmaxf(v, -65504.0f), 65504.0f);
+  return __float2half_rn(v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
+  return __uint_as_float(bits16 << 16);
+}
+
+// ------------------------------------------------------------- tensor cores
+// D += A * B, m16n8k16, f16 inputs, f32 accumulators (legacy warp-level MMA;
+// used for the bandwidth-bound decode GEMVs where the MMA pipe is not the
+// bottleneck).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------------- memory
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t ldg_nc_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float gelu_tanh(float g) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2 / pi)
+  const float k1 = 0.044715f;
+  return 0.5f * g * (1.0f + tanhf(k0 * (g + k1 * g * g * g)));
+}
+
+}  // namespace nvfp4moe

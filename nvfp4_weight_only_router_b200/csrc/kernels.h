@@ -1,0 +1,72 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4moe {
+
+cudaError_t launch_quantize(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* q,
+                            uint8_t* s, float* g, uint32_t* amax_ws, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* q, const uint8_t* s, const float* g, int64_t E,
+                              int64_t N, int64_t K, float* out, cudaStream_t st);
+
+struct RouteArgs {
+  const uint16_t* x;      // bf16 [T, H]
+  const uint16_t* proj;   // bf16 [E, H]
+  const uint16_t* scale;  // bf16 [H]
+  const uint16_t* pes;    // bf16 [E]
+  const float* bias;      // f32 [E] or null
+  int T, H, ksplit, segs_per_split;
+  float eps, inv_sqrt_h;
+  float* part_logits;     // [ksplit, T, 128]
+  float* part_ss;         // [ksplit, T]
+  int* tile_counter;      // [ceil(T/16)], zero on entry, left zero
+  int32_t* ids;           // [T, 8]
+  float* wts;             // [T, 8]
+  __half* x16;            // optional f16 copy of x [T, H]
+  int* status;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+
+struct PermuteArgs {
+  const int32_t* ids;  // [S]
+  int S, nchunks;
+  int* meta;           // kMetaInts ints (counter zero on entry, left zero)
+  int* chunk_count;    // [nchunks, 128]
+  int* chunk_base;     // [nchunks, 128]
+  int* local_rank;     // [S]
+  int* sorted_slot;    // [S]
+  int* slot_pos;       // [S]
+  int* status;
+};
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
+
+struct ExpertArgs {
+  const uint8_t* gu_q;
+  const uint8_t* gu_s;
+  const float* gu_g;
+  const uint8_t* dn_q;
+  const uint8_t* dn_s;
+  const float* dn_g;
+  const __half* x16;        // [T, H]
+  const int* meta;
+  const int* sorted_slot;   // [S]
+  const int* slot_pos;      // [S]
+  const float* wts;         // [S]
+  __half* h;                // [S, I], rows in sorted order
+  float* obuf;              // mode 0: [S, H] per-slot outputs, sorted order
+  float* yacc;              // mode 1: [T, H] fp32 accumulator (zero on entry)
+  void* y;                  // bf16 [T, H]
+  int T, max_active, mode;
+  int* status;
+};
+cudaError_t launch_gate_up_gemv(const ExpertArgs& a, cudaStream_t st);
+cudaError_t launch_down_gemv(const ExpertArgs& a, cudaStream_t st);
+cudaError_t launch_finalize(const ExpertArgs& a, cudaStream_t st);
+
+cudaError_t launch_residual_rmsnorm(float* res, const uint16_t* y, uint16_t* x_out, int T, int H,
+                                    float eps, cudaStream_t st);
+
+}  // namespace nvfp4moe

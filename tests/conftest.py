@@ -29,3 +29,25 @@ def golden_lines(name):
 @pytest.fixture(scope="session")
 def golden():
     return golden_lines
+
+
+@pytest.fixture(scope="session")
+def dev():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from nvfp4_weight_only_router_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+    return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def layer0(dev):
+    """The decode/prefill layer: experts seed 0, router seed 1 (host copies and
+    device copies)."""
+    import moe_inputs as gen
+    import nvfp4_weight_only_router_b200 as lib
+    ex = gen.make_experts(0)
+    rt = gen.make_router(1)
+    return {"ex": ex, "rt": rt, "dex": lib.Experts.from_host(ex, dev), "drt": lib.Router.from_host(rt, dev)}

@@ -1,0 +1,116 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects invalid arguments with the documented status
+codes before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def capi():
+    from nvfp4_weight_only_router_b200 import build
+    build.build()
+    from nvfp4_weight_only_router_b200 import capi
+    return capi
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "nvfp4moe.h")).read()
+    return re.findall(r"NVFP4MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+def test_every_declared_symbol_is_exported(capi):
+    names = header_functions()
+    assert len(names) == 13
+    for n in names:
+        assert hasattr(capi.lib, n), n
+        assert n in capi.SIGNATURES, n
+
+
+def test_only_declared_symbols_are_exported(capi):
+    out = os.popen(f"nm -D --defined-only {capi.LIB_PATH}").read().split("\n")
+    exported = {l.split()[-1] for l in out if " T " in l}
+    assert exported == set(header_functions())
+
+
+def test_abi_version_and_status_strings(capi):
+    assert capi.nvfp4_abi_version() == 1
+    for code in range(8):
+        assert capi.status_string(code)
+    assert capi.status_string(0) == "ok"
+
+
+def _router(capi, E=128, H=2816, k=8, eps=1e-6, ptr=4096):
+    return capi.moe_router(ptr, ptr, ptr, None, E, H, k, eps)
+
+
+def _experts(capi, E=128, H=2816, I=704, ptr=4096):
+    return capi.moe_experts(ptr, ptr, ptr, ptr, ptr, ptr, E, H, I)
+
+
+def test_quantize_validation(capi):
+    c = capi
+    assert c.nvfp4_quantize_workspace_bytes(128, 1408, 2816) == 512
+    assert c.nvfp4_quantize_workspace_bytes(0, 1, 32) == 0
+    P = 4096
+    assert c.nvfp4_quantize(None, 1, 16, 32, P, P, P, P, 256, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.nvfp4_quantize(P, 1, 16, 24, P, P, P, P, 256, None) == c.NVFP4_ERR_UNSUPPORTED
+    assert c.nvfp4_quantize(P, 0, 16, 32, P, P, P, P, 256, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.nvfp4_quantize(P + 8, 1, 16, 32, P, P, P, P, 256, None) == c.NVFP4_ERR_ALIGNMENT
+    assert c.nvfp4_quantize(P, 1, 16, 32, P, P, P, None, 256, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.nvfp4_quantize(P, 1, 16, 32, P, P, P, P, 0, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.nvfp4_quantize(P, 1, 16, 32, P, P, P, P + 16, 4096, None) == c.NVFP4_ERR_ALIGNMENT
+    assert c.nvfp4_quantize(P, 1, 1 << 20, 4096, P, P, P, P, 4096, None) == c.NVFP4_ERR_UNSUPPORTED
+
+
+def test_route_validation(capi):
+    c = capi
+    r = _router(c)
+    assert c.moe_route_workspace_bytes(1, ctypes.byref(r)) > 0
+    assert c.moe_route_workspace_bytes(0, ctypes.byref(r)) == 0
+    assert c.moe_route_workspace_bytes(65537, ctypes.byref(r)) == 0
+    P = 4096
+    assert c.moe_route(P, 1, ctypes.byref(r), P, P, None, 0, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.moe_route(None, 1, ctypes.byref(r), P, P, P, 1 << 20, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_route(P, 0, ctypes.byref(r), P, P, P, 1 << 20, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_route(P, 1, None, P, P, P, 1 << 20, None) == c.NVFP4_ERR_INVALID_ARG
+    for bad, code in [(_router(c, E=64), c.NVFP4_ERR_UNSUPPORTED), (_router(c, k=4), c.NVFP4_ERR_UNSUPPORTED),
+                      (_router(c, H=100), c.NVFP4_ERR_UNSUPPORTED), (_router(c, eps=-1.0), c.NVFP4_ERR_INVALID_ARG),
+                      (_router(c, ptr=4097), c.NVFP4_ERR_ALIGNMENT)]:
+        assert c.moe_route(P, 1, ctypes.byref(bad), P, P, P, 1 << 20, None) == code
+    assert c.moe_route(P + 2, 1, ctypes.byref(r), P, P, P, 1 << 20, None) == c.NVFP4_ERR_ALIGNMENT
+    assert c.moe_route(P, 1, ctypes.byref(r), P, P, P + 16, 1 << 20, None) == c.NVFP4_ERR_ALIGNMENT
+
+
+def test_forward_validation_and_workspace_sizes(capi):
+    c = capi
+    r, x = _router(c), _experts(c)
+    sizes = [c.moe_forward_workspace_bytes(T, ctypes.byref(x), ctypes.byref(r)) for T in (1, 64, 4096)]
+    assert 0 < sizes[0] < sizes[1] < sizes[2]
+    assert sizes[2] < 1 << 31
+    assert c.moe_forward_workspace_bytes(1, ctypes.byref(_experts(c, I=512)), ctypes.byref(r)) == 0
+    P = 4096
+    ws = sizes[0]
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(x), ctypes.byref(r), P, P, ws - 1, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.moe_nvfp4_forward(None, 1, ctypes.byref(x), ctypes.byref(r), P, P, ws, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(x), ctypes.byref(r), None, P, ws, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(_experts(c, H=2048)), ctypes.byref(r), P, P, ws, None) == c.NVFP4_ERR_UNSUPPORTED
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(x), ctypes.byref(_router(c, H=2048)), P, P, ws, None) == c.NVFP4_ERR_UNSUPPORTED
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(_experts(c, ptr=4100)), ctypes.byref(r), P, P, ws, None) == c.NVFP4_ERR_ALIGNMENT
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(x), ctypes.byref(r), P, P + 128, ws, None) == c.NVFP4_ERR_ALIGNMENT
+    v = c.moe_forward_views()
+    assert c.moe_forward_workspace_views(64, ctypes.byref(x), ctypes.byref(r), ctypes.byref(v)) == 0
+    offs = [v.ids, v.weights, v.counts, v.offsets, v.sorted_slot, v.slot_pos, v.h]
+    assert all(o % 4 == 0 for o in offs) and max(offs) < sizes[1]
+
+
+def test_residual_validation(capi):
+    c = capi
+    P = 4096
+    assert c.moe_residual_rmsnorm(None, None, P, 1, 2816, 1e-6, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_residual_rmsnorm(P, None, P, 1, 2817, 1e-6, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_residual_rmsnorm(P + 4, None, P, 1, 2816, 1e-6, None) == c.NVFP4_ERR_ALIGNMENT

@@ -1,0 +1,52 @@
+"""moe_route on the GPU against the oracle router (fp64)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as gen
+import nvfp4_weight_only_router_b200 as lib
+from oracle import moe as M
+from tests.gpu_common import bf16_to_dev, check_ids, check_weights
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(x, rt, drt, dev):
+    ids, w = lib.route(bf16_to_dev(x, dev), drt)
+    torch.cuda.synchronize()
+    ids, w = ids.cpu().numpy(), w.cpu().numpy()
+    ids0, w0, logits = M.route(x, rt)
+    differ = check_ids(ids, ids0, logits)
+    check_weights(w, w0, differ)
+    return differ
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 17, 64, 257, 300])
+def test_route_layer_router(layer0, dev, T):
+    x = gen.make_x(100 + T, T)
+    _check(x, layer0["rt"], layer0["drt"], dev)
+
+
+def test_route_prefill_zipf_bias(dev):
+    rt = gen.make_router(1, bias=gen.zipf_bias(7))
+    drt = lib.Router.from_host(rt, dev)
+    x = gen.make_x(2, 4096)
+    differ = _check(x, rt, drt, dev)
+    assert differ.mean() < 1e-3
+
+
+def test_route_other_hidden_size(dev):
+    rt = gen.make_router(5, h=256)
+    drt = lib.Router.from_host(rt, dev)
+    x = gen.make_x(6, 33, 256)
+    _check(x, rt, drt, dev)
+
+
+def test_route_ties_pick_lower_id(dev):
+    # identical router rows -> identical logits; top-8 must be the lowest ids
+    rt = gen.make_router(8)
+    rt.proj[:] = rt.proj[0]
+    drt = lib.Router.from_host(rt, dev)
+    x = gen.make_x(9, 4)
+    ids, _ = lib.route(bf16_to_dev(x, dev), drt)
+    assert (ids.cpu().numpy() == np.arange(8)[None, :]).all()
