@@ -289,7 +289,7 @@ def run_ours(args, wl, rank, world, local_rank):
 
     # -------- warm-up (at least W steps and at least 1 s, so the clock sampler sees load)
     sampler = ClockSampler(physical_gpu_index(local_rank))
-    t_end = time.perf_counter() + 1.0
+    t_end = time.perf_counter() + args.min_warmup_s
     i = 0
     while i < args.warmup or time.perf_counter() < t_end:
         if args.workload != "quantize":
@@ -429,6 +429,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode64", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-warmup-s", type=float, default=1.0,
+                    help="keep warming up for at least this long (the clock sampler needs load)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", "0"))

@@ -282,8 +282,16 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
   cudaStream_t s = as_stream(stream);
   int* status = device_status_ptr();
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (ev && cudaStreamIsCapturing(s, &cap) != cudaSuccess) return NVFP4_ERR_CUDA;
   auto mark = [&](int i) -> bool {
-    return !ev || !ev[i] || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
+    if (!ev || !ev[i]) return true;
+    cudaEvent_t e = static_cast<cudaEvent_t>(ev[i]);
+    // inside a stream capture, an external record becomes an event-record node
+    // of the graph (a plain record would only order the capture)
+    if (cap == cudaStreamCaptureStatusActive)
+      return cudaEventRecordWithFlags(e, s, cudaEventRecordExternal) == cudaSuccess;
+    return cudaEventRecord(e, s) == cudaSuccess;
   };
   if (!mark(0)) return NVFP4_ERR_CUDA;
 
