@@ -119,6 +119,25 @@ NVFP4MOE_API nvfp4_status nvfp4_quantize(const void* w_dev, int64_t E, int64_t N
                             uint8_t* q_dev, uint8_t* s_dev, float* g_dev,
                             void* ws_dev, size_t ws_bytes, void* stream);
 
+/* nvfp4_quantize_noalloc: nvfp4_quantize for callers that cannot allocate
+ * device memory when they quantise -- for instance a plugin whose host
+ * framework owns all device memory and forbids allocation inside its execute
+ * callback, or a latency-critical path that must not enter an allocator.  It
+ * takes no workspace: the per-tensor amax scratch lives in a fixed 16 KiB
+ * device array inside the library (held on every GPU that loads the library
+ * until the process exits), and the call allocates nothing (no cudaMalloc,
+ * no allocating library routine).  The pages have no counterpart of this
+ * entry point; it exists for such callers only.
+ * Same arguments, layouts, results and limits as nvfp4_quantize, plus
+ * E <= 4096 (NVFP4_ERR_UNSUPPORTED beyond).  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress, with that device
+ * current); make that first call before any stream capture.  All calls on a
+ * device share the array, which keeps the last call's contents (each call
+ * clears what it needs): calls that overlap on the GPU race. */
+NVFP4MOE_API nvfp4_status nvfp4_quantize_noalloc(const void* w_dev, int64_t E, int64_t N, int64_t K,
+                                                 uint8_t* q_dev, uint8_t* s_dev, float* g_dev,
+                                                 void* stream);
+
 /* nvfp4_dequantize: w = e2m1 * e4m3 * G rounded once to fp32 ("Gemma-4-26B-A4B-
  * NVFP4-mlx", "Quantization recipe": E2M1 x per-16 E4M3 x per-tensor F32).
  * Same layouts and limits as nvfp4_quantize; out_dev f32 [E, N, K].  No

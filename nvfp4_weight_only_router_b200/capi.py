@@ -59,6 +59,8 @@ SIGNATURES = {
     "nvfp4_quantize_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int64]),
     "nvfp4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_size_t, c_void_p]),
+    "nvfp4_quantize_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p,
+                                         c_void_p, c_void_p]),
     "nvfp4_dequantize": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64,
                                    c_void_p, c_void_p]),
     "moe_route_workspace_bytes": (c_size_t, [c_int32, _R]),
