@@ -51,26 +51,21 @@ struct Alloc {
 };
 
 struct RouteLayout {
-  int ntiles = 0, ksplit = 0, segs_per_split = 0;
-  Region counters, part_logits, part_ss;
+  int ntiles = 0;
+  bool few_tokens = false;
+  Region counters, logits;
 };
 
-RouteLayout route_layout(Alloc& al, int T, int H) {
+RouteLayout route_layout(Alloc& al, int T) {
   RouteLayout L;
   L.ntiles = (T + 15) / 16;
-  const int nseg = H / kSegK;
-  if (T <= 256) {
-    L.ksplit = nseg;
-    L.segs_per_split = 1;
-  } else {
-    L.ksplit = 1;
-    L.segs_per_split = nseg;
-  }
+  L.few_tokens = T <= 256;
   L.counters = al.take(sizeof(int) * L.ntiles);
-  L.part_logits = al.take(sizeof(float) * (size_t)L.ksplit * T * kE);
-  L.part_ss = al.take(sizeof(float) * (size_t)L.ksplit * T);
+  L.logits = al.take(sizeof(float) * (size_t)T * kE);
   return L;
 }
+
+constexpr int kFusedPermuteMaxSlots = 1024;  // the router's last CTA groups the slots
 
 struct FwdLayout {
   Region meta;
@@ -90,7 +85,7 @@ FwdLayout fwd_layout(int T) {
   L.mode = (T <= kDeterministicMaxT) ? 0 : 1;
   // zeroed on entry: meta (includes the permute counter) and the router counters
   L.meta = al.take(sizeof(int) * kMetaInts);
-  L.route = route_layout(al, T, kH);
+  L.route = route_layout(al, T);
   L.ids = al.take(sizeof(int) * L.S);
   L.wts = al.take(sizeof(float) * L.S);
   L.chunk_count = al.take(sizeof(int) * (size_t)L.nchunks * kE);
@@ -149,16 +144,17 @@ RouteArgs make_route_args(const void* x, int T, const moe_router* r, const Route
   a.bias = r->logit_bias;
   a.T = T;
   a.H = r->H;
-  a.ksplit = L.ksplit;
-  a.segs_per_split = L.segs_per_split;
+  a.few_tokens = L.few_tokens;
   a.eps = r->eps;
   a.inv_sqrt_h = (float)(1.0 / std::sqrt((double)r->H));
-  a.part_logits = at<float>(ws, L.part_logits);
-  a.part_ss = at<float>(ws, L.part_ss);
+  a.logits = at<float>(ws, L.logits);
   a.tile_counter = at<int>(ws, L.counters);
   a.ids = ids;
   a.wts = wts;
   a.x16 = x16;
+  a.meta = nullptr;
+  a.sorted_slot = nullptr;
+  a.slot_pos = nullptr;
   a.status = status;
   return a;
 }
@@ -223,7 +219,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* s, const float* g
 size_t moe_route_workspace_bytes(int32_t T, const moe_router* r) {
   if (T < 1 || T > 65536 || check_router(r, false) != NVFP4_OK) return 0;
   Alloc al;
-  route_layout(al, T, r->H);
+  route_layout(al, T);
   return al.cur;
 }
 
@@ -237,7 +233,7 @@ nvfp4_status moe_route(const void* x, int32_t T, const moe_router* r, int32_t* i
   if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
   Alloc al;
-  RouteLayout L = route_layout(al, T, r->H);
+  RouteLayout L = route_layout(al, T);
   cudaStream_t s = as_stream(stream);
   cudaError_t e = cudaMemsetAsync(at<int>(ws, L.counters), 0, L.counters.bytes, s);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -305,6 +301,12 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   float* wts = at<float>(ws, L.wts);
   __half* x16 = at<__half>(ws, L.x16);
   RouteArgs ra = make_route_args(x, T, r, L.route, ws, ids, wts, x16, status);
+  const bool fused_permute = L.S <= kFusedPermuteMaxSlots;
+  if (fused_permute) {
+    ra.meta = at<int>(ws, L.meta);
+    ra.sorted_slot = at<int>(ws, L.sorted);
+    ra.slot_pos = at<int>(ws, L.pos);
+  }
   if ((e = launch_route(ra, s)) != cudaSuccess || !mark(1)) return NVFP4_ERR_CUDA;
 
   PermuteArgs pa;
@@ -318,7 +320,8 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   pa.sorted_slot = at<int>(ws, L.sorted);
   pa.slot_pos = at<int>(ws, L.pos);
   pa.status = status;
-  if ((e = launch_permute(pa, s)) != cudaSuccess || !mark(2)) return NVFP4_ERR_CUDA;
+  if (!fused_permute && (e = launch_permute(pa, s)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (!mark(2)) return NVFP4_ERR_CUDA;
 
   ExpertArgs xa;
   xa.gu_q = ex->gate_up_q;
@@ -340,8 +343,11 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   xa.max_active = L.S < kE ? L.S : kE;
   xa.mode = L.mode;
   xa.status = status;
-  if ((e = launch_gate_up_gemv(xa, s)) != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
-  if ((e = launch_down_gemv(xa, s)) != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
+  const bool stream_path = L.mode == 0;  // few tokens per expert: bandwidth-bound streaming GEMV
+  e = stream_path ? launch_gate_up_stream(xa, s) : launch_gate_up_tc(xa, s);
+  if (e != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
+  e = stream_path ? launch_down_stream(xa, s) : launch_down_tc(xa, s);
+  if (e != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
   if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return NVFP4_ERR_CUDA;
   return NVFP4_OK;
 }

@@ -18,14 +18,19 @@ struct RouteArgs {
   const uint16_t* scale;  // bf16 [H]
   const uint16_t* pes;    // bf16 [E]
   const float* bias;      // f32 [E] or null
-  int T, H, ksplit, segs_per_split;
+  int T, H;
+  bool few_tokens;        // 16 CTAs of 8 experts per token tile (else 1 CTA of 128)
   float eps, inv_sqrt_h;
-  float* part_logits;     // [ksplit, T, 128]
-  float* part_ss;         // [ksplit, T]
+  float* logits;          // [T, 128] scratch
   int* tile_counter;      // [ceil(T/16)], zero on entry, left zero
   int32_t* ids;           // [T, 8]
   float* wts;             // [T, 8]
   __half* x16;            // optional f16 copy of x [T, H]
+  // optional fused permutation (T*8 <= 1024): meta (route counter zero on
+  // entry), sorted_slot [T*8], slot_pos [T*8]; meta == null -> not fused
+  int* meta;
+  int* sorted_slot;
+  int* slot_pos;
   int* status;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
@@ -65,6 +70,12 @@ struct ExpertArgs {
 cudaError_t launch_gate_up_gemv(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_down_gemv(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_finalize(const ExpertArgs& a, cudaStream_t st);
+// persistent bulk-copy streaming versions (decode: few tokens per expert)
+cudaError_t launch_gate_up_stream(const ExpertArgs& a, cudaStream_t st);
+cudaError_t launch_down_stream(const ExpertArgs& a, cudaStream_t st);
+// tcgen05 grouped GEMMs (many tokens per expert)
+cudaError_t launch_gate_up_tc(const ExpertArgs& a, cudaStream_t st);
+cudaError_t launch_down_tc(const ExpertArgs& a, cudaStream_t st);
 
 cudaError_t launch_residual_rmsnorm(float* res, const uint16_t* y, uint16_t* x_out, int T, int H,
                                     float eps, cudaStream_t st);
