@@ -1,6 +1,7 @@
 // C ABI of the NVFP4 MoE library: argument validation, workspace layout and
 // launch sequencing on the caller's stream.  See include/nvfp4moe.h.
 #include <cmath>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/nvfp4moe.h"
@@ -67,22 +68,31 @@ RouteLayout route_layout(Alloc& al, int T) {
 
 constexpr int kFusedPermuteMaxSlots = 1024;  // the router's last CTA groups the slots
 
+// Largest token count that takes the streaming GEMV path; above it the
+// tensor-core grouped GEMMs run.  NVFP4MOE_STREAM_MAX_T overrides the default
+// (read once per process) so the crossover can be re-measured.
+int stream_max_tokens() {
+  static const int v = [] {
+    const char* e = std::getenv("NVFP4MOE_STREAM_MAX_T");
+    return e ? std::atoi(e) : 256;
+  }();
+  return v;
+}
+
 struct FwdLayout {
   Region meta;
   RouteLayout route;
-  Region ids, wts, chunk_count, chunk_base, local_rank, sorted, pos, x16, h, obuf, yacc;
-  int S = 0, nchunks = 0, mode = 0;
+  Region ids, wts, chunk_count, chunk_base, local_rank, sorted, pos, x16, xs, h, obuf;
+  int S = 0, nchunks = 0;
   size_t total = 0;
 };
 
-constexpr int kDeterministicMaxT = 256;  // per-slot combine buffer up to this T
 
 FwdLayout fwd_layout(int T) {
   FwdLayout L;
   Alloc al;
   L.S = T * kTopK;
   L.nchunks = (L.S + 1023) / 1024;
-  L.mode = (T <= kDeterministicMaxT) ? 0 : 1;
   // zeroed on entry: meta (includes the permute counter) and the router counters
   L.meta = al.take(sizeof(int) * kMetaInts);
   L.route = route_layout(al, T);
@@ -94,11 +104,10 @@ FwdLayout fwd_layout(int T) {
   L.sorted = al.take(sizeof(int) * L.S);
   L.pos = al.take(sizeof(int) * L.S);
   L.x16 = al.take(sizeof(__half) * (size_t)T * kH);
+  L.xs = al.take(sizeof(__half) * (size_t)L.S * kH);
   L.h = al.take(sizeof(__half) * (size_t)L.S * kI);
-  if (L.mode == 0)
-    L.obuf = al.take(sizeof(float) * (size_t)L.S * kH);
-  else
-    L.yacc = al.take(sizeof(float) * (size_t)T * kH);
+  // per-slot outputs, summed in slot order by the combine: deterministic
+  L.obuf = al.take(sizeof(float) * (size_t)L.S * kH);
   L.total = al.cur;
   return L;
 }
@@ -294,7 +303,6 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   // meta and router counters are contiguous at the start of the workspace
   const size_t zero_bytes = L.route.counters.off + L.route.counters.bytes;
   cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, s);
-  if (e == cudaSuccess && L.mode == 1) e = cudaMemsetAsync(at<float>(ws, L.yacc), 0, L.yacc.bytes, s);
   if (e != cudaSuccess) return NVFP4_ERR_CUDA;
 
   int32_t* ids = at<int32_t>(ws, L.ids);
@@ -336,18 +344,28 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   xa.slot_pos = pa.slot_pos;
   xa.wts = wts;
   xa.h = at<__half>(ws, L.h);
-  xa.obuf = L.mode == 0 ? at<float>(ws, L.obuf) : nullptr;
-  xa.yacc = L.mode == 1 ? at<float>(ws, L.yacc) : nullptr;
+  xa.obuf = at<float>(ws, L.obuf);
   xa.y = y;
   xa.T = T;
   xa.max_active = L.S < kE ? L.S : kE;
-  xa.mode = L.mode;
   xa.status = status;
-  const bool stream_path = L.mode == 0;  // few tokens per expert: bandwidth-bound streaming GEMV
-  e = stream_path ? launch_gate_up_stream(xa, s) : launch_gate_up_tc(xa, s);
-  if (e != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
-  e = stream_path ? launch_down_stream(xa, s) : launch_down_tc(xa, s);
-  if (e != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
+  xa.xs = at<__half>(ws, L.xs);
+  if (T <= stream_max_tokens()) {
+    // few tokens per expert: the weight stream bounds the step, so a
+    // bandwidth-bound GEMV that reads x and h in place is fastest
+    e = launch_gate_up_stream(xa, s);
+    if (e != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
+    e = launch_down_stream(xa, s);
+    if (e != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
+  } else {
+    // many tokens per expert: tensor-core grouped GEMMs on expert-sorted rows
+    const int nt = T <= 512 ? 64 : 192;  // about the tokens an expert gets
+    if ((e = launch_gather_sorted(xa, s)) != cudaSuccess) return NVFP4_ERR_CUDA;
+    e = launch_moe_gate_up(xa, nt, s);
+    if (e != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
+    e = launch_moe_down(xa, nt, s);
+    if (e != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
+  }
   if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return NVFP4_ERR_CUDA;
   return NVFP4_OK;
 }

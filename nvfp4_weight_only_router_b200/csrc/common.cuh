@@ -134,10 +134,16 @@ __device__ __forceinline__ uint16_t ldg_nc_u16(const void* p) {
   return v;
 }
 
+// GELU, tanh form: 0.5 g (1 + tanh(a)), a = sqrt(2/pi) (g + 0.044715 g^3),
+// evaluated through the identity 0.5 (1 + tanh(a)) = 1 / (1 + exp(-2a)).
+// The exponential (__expf, relative error ~2^-21) keeps the result within a
+// few fp32 ulps of the tanh expression; exp overflow for very negative g gives
+// the correct limit 0.
 __device__ __forceinline__ float gelu_tanh(float g) {
   const float k0 = 0.7978845608028654f;  // sqrt(2 / pi)
   const float k1 = 0.044715f;
-  return 0.5f * g * (1.0f + tanhf(k0 * (g + k1 * g * g * g)));
+  const float a = k0 * (g + k1 * g * g * g);
+  return g / (1.0f + __expf(-2.0f * a));
 }
 
 }  // namespace nvfp4moe

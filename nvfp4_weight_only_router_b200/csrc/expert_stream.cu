@@ -325,14 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1) stream_gemv_kernel(ExpertArgs p) 
             const int slot = p.sorted_slot[pos];
             const float wgt = p.wts[slot] * G;
             const float o0 = vv[c] * wgt, o1 = vv[2 + c] * wgt;
-            if (p.mode == 0) {
-              p.obuf[(size_t)pos * kH + row0] = o0;
-              p.obuf[(size_t)pos * kH + row0 + 8] = o1;
-            } else {
-              const int tok = slot / kTopK;
-              atomicAdd(p.yacc + (size_t)tok * kH + row0, o0);
-              atomicAdd(p.yacc + (size_t)tok * kH + row0 + 8, o1);
-            }
+            p.obuf[(size_t)pos * kH + row0] = o0;
+            p.obuf[(size_t)pos * kH + row0 + 8] = o1;
           }
         }
       }

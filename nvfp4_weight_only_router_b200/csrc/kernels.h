@@ -56,26 +56,27 @@ struct ExpertArgs {
   const uint8_t* dn_s;
   const float* dn_g;
   const __half* x16;        // [T, H]
+  __half* xs;               // [S, H] activations in expert-sorted slot order
   const int* meta;
   const int* sorted_slot;   // [S]
   const int* slot_pos;      // [S]
   const float* wts;         // [S]
   __half* h;                // [S, I], rows in sorted order
-  float* obuf;              // mode 0: [S, H] per-slot outputs, sorted order
-  float* yacc;              // mode 1: [T, H] fp32 accumulator (zero on entry)
+  float* obuf;              // [S, H] per-slot weighted outputs, sorted order
   void* y;                  // bf16 [T, H]
-  int T, max_active, mode;
+  int T, max_active;
   int* status;
 };
-cudaError_t launch_gate_up_gemv(const ExpertArgs& a, cudaStream_t st);
-cudaError_t launch_down_gemv(const ExpertArgs& a, cudaStream_t st);
+// y[t] = bf16(sum over the token's 8 slots of obuf, in slot order)
 cudaError_t launch_finalize(const ExpertArgs& a, cudaStream_t st);
 // persistent bulk-copy streaming versions (decode: few tokens per expert)
 cudaError_t launch_gate_up_stream(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_down_stream(const ExpertArgs& a, cudaStream_t st);
-// tcgen05 grouped GEMMs (many tokens per expert)
-cudaError_t launch_gate_up_tc(const ExpertArgs& a, cudaStream_t st);
-cudaError_t launch_down_tc(const ExpertArgs& a, cudaStream_t st);
+// tcgen05 grouped GEMMs with the dequantised weights in tensor memory;
+// nt = tokens per tile (16, 64 or 192)
+cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st);
+cudaError_t launch_moe_gate_up(const ExpertArgs& a, int nt, cudaStream_t st);
+cudaError_t launch_moe_down(const ExpertArgs& a, int nt, cudaStream_t st);
 
 cudaError_t launch_residual_rmsnorm(float* res, const uint16_t* y, uint16_t* x_out, int T, int H,
                                     float eps, cudaStream_t st);
