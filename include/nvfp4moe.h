@@ -230,6 +230,11 @@ NVFP4MOE_API nvfp4_status nvfp4_get_device_status(void* stream);
 NVFP4MOE_API const char* nvfp4_status_string(nvfp4_status status);
 NVFP4MOE_API int nvfp4_abi_version(void);
 
+/* The CUDA runtime's text for the error behind the last NVFP4_ERR_CUDA that a
+ * call of this library returned on the calling thread ("no error" if none).
+ * A static string owned by the CUDA runtime; never NULL. */
+NVFP4MOE_API const char* nvfp4_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

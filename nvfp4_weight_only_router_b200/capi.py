@@ -74,6 +74,7 @@ SIGNATURES = {
     "nvfp4_get_device_status": (c_int32, [c_void_p]),
     "nvfp4_status_string": (ctypes.c_char_p, [c_int32]),
     "nvfp4_abi_version": (ctypes.c_int, []),
+    "nvfp4_last_cuda_error": (ctypes.c_char_p, []),
 }
 
 for _name, (_res, _args) in SIGNATURES.items():
@@ -86,7 +87,10 @@ for _name, (_res, _args) in SIGNATURES.items():
 class NVFP4Error(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
-        super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
+        msg = f"{what}: {STATUS.get(status, status)} ({status_string(status)})"
+        if status == NVFP4_ERR_CUDA:
+            msg += f": {lib.nvfp4_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 def status_string(status: int) -> str:

@@ -117,7 +117,15 @@ T* at(void* ws, const Region& r) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + r.off);
 }
 
-nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+// the last CUDA error behind an NVFP4_ERR_CUDA status, per calling thread
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+nvfp4_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = e != cudaSuccess ? e : cudaErrorUnknown;
+  return NVFP4_ERR_CUDA;
+}
+
+nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : cuda_fail(e); }
 
 nvfp4_status check_router(const moe_router* r, bool forward) {
   if (!r || !r->proj || !r->scale || !r->per_expert_scale) return NVFP4_ERR_INVALID_ARG;
@@ -173,6 +181,8 @@ RouteArgs make_route_args(const void* x, int T, const moe_router* r, const Route
 extern "C" {
 
 int nvfp4_abi_version(void) { return NVFP4MOE_ABI_VERSION; }
+
+const char* nvfp4_last_cuda_error(void) { return cudaGetErrorString(t_last_cuda_error); }
 
 const char* nvfp4_status_string(nvfp4_status s) {
   switch (s) {
@@ -245,7 +255,7 @@ nvfp4_status moe_route(const void* x, int32_t T, const moe_router* r, int32_t* i
   RouteLayout L = route_layout(al, T);
   cudaStream_t s = as_stream(stream);
   cudaError_t e = cudaMemsetAsync(at<int>(ws, L.counters), 0, L.counters.bytes, s);
-  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   RouteArgs a = make_route_args(x, T, r, L, ws, ids, w, nullptr, device_status_ptr());
   return cuda_status(launch_route(a, s));
 }
@@ -288,7 +298,7 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   cudaStream_t s = as_stream(stream);
   int* status = device_status_ptr();
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-  if (ev && cudaStreamIsCapturing(s, &cap) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (ev && cudaStreamIsCapturing(s, &cap) != cudaSuccess) return cuda_fail(cudaGetLastError());
   auto mark = [&](int i) -> bool {
     if (!ev || !ev[i]) return true;
     cudaEvent_t e = static_cast<cudaEvent_t>(ev[i]);
@@ -298,12 +308,12 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
       return cudaEventRecordWithFlags(e, s, cudaEventRecordExternal) == cudaSuccess;
     return cudaEventRecord(e, s) == cudaSuccess;
   };
-  if (!mark(0)) return NVFP4_ERR_CUDA;
+  if (!mark(0)) return cuda_fail(cudaGetLastError());
 
   // meta and router counters are contiguous at the start of the workspace
   const size_t zero_bytes = L.route.counters.off + L.route.counters.bytes;
   cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, s);
-  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
 
   int32_t* ids = at<int32_t>(ws, L.ids);
   float* wts = at<float>(ws, L.wts);
@@ -315,7 +325,7 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
     ra.sorted_slot = at<int>(ws, L.sorted);
     ra.slot_pos = at<int>(ws, L.pos);
   }
-  if ((e = launch_route(ra, s)) != cudaSuccess || !mark(1)) return NVFP4_ERR_CUDA;
+  if ((e = launch_route(ra, s)) != cudaSuccess || !mark(1)) return cuda_fail(e);
 
   PermuteArgs pa;
   pa.ids = ids;
@@ -328,8 +338,8 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   pa.sorted_slot = at<int>(ws, L.sorted);
   pa.slot_pos = at<int>(ws, L.pos);
   pa.status = status;
-  if (!fused_permute && (e = launch_permute(pa, s)) != cudaSuccess) return NVFP4_ERR_CUDA;
-  if (!mark(2)) return NVFP4_ERR_CUDA;
+  if (!fused_permute && (e = launch_permute(pa, s)) != cudaSuccess) return cuda_fail(e);
+  if (!mark(2)) return cuda_fail(cudaGetLastError());
 
   ExpertArgs xa;
   xa.gu_q = ex->gate_up_q;
@@ -350,23 +360,23 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   xa.max_active = L.S < kE ? L.S : kE;
   xa.status = status;
   xa.xs = at<__half>(ws, L.xs);
+  if ((e = launch_gather_sorted(xa, s)) != cudaSuccess) return cuda_fail(e);
   if (T <= stream_max_tokens()) {
-    // few tokens per expert: the weight stream bounds the step, so a
-    // bandwidth-bound GEMV that reads x and h in place is fastest
+    // few tokens per expert: the weight stream bounds the step (streaming
+    // GEMV with register dequantisation)
     e = launch_gate_up_stream(xa, s);
-    if (e != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
+    if (e != cudaSuccess || !mark(3)) return cuda_fail(e);
     e = launch_down_stream(xa, s);
-    if (e != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
+    if (e != cudaSuccess || !mark(4)) return cuda_fail(e);
   } else {
     // many tokens per expert: tensor-core grouped GEMMs on expert-sorted rows
     const int nt = T <= 512 ? 64 : 192;  // about the tokens an expert gets
-    if ((e = launch_gather_sorted(xa, s)) != cudaSuccess) return NVFP4_ERR_CUDA;
     e = launch_moe_gate_up(xa, nt, s);
-    if (e != cudaSuccess || !mark(3)) return NVFP4_ERR_CUDA;
+    if (e != cudaSuccess || !mark(3)) return cuda_fail(e);
     e = launch_moe_down(xa, nt, s);
-    if (e != cudaSuccess || !mark(4)) return NVFP4_ERR_CUDA;
+    if (e != cudaSuccess || !mark(4)) return cuda_fail(e);
   }
-  if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return NVFP4_ERR_CUDA;
+  if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return cuda_fail(e);
   return NVFP4_OK;
 }
 
@@ -396,12 +406,12 @@ nvfp4_status moe_residual_rmsnorm(float* res, const void* y, void* x_out, int32_
 // ----------------------------------------------------------- device status
 nvfp4_status nvfp4_get_device_status(void* stream) {
   int* p = device_status_ptr();
-  if (!p) return NVFP4_ERR_CUDA;
+  if (!p) return cuda_fail(cudaGetLastError());
   cudaStream_t s = as_stream(stream);
   int v = 0;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return NVFP4_ERR_CUDA;
-  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NVFP4_ERR_CUDA;
-  if (v != 0 && cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return cuda_fail(cudaGetLastError());
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return cuda_fail(cudaGetLastError());
+  if (v != 0 && cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return cuda_fail(cudaGetLastError());
   return static_cast<nvfp4_status>(v);
 }
 

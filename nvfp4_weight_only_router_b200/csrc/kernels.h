@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -69,7 +70,7 @@ struct ExpertArgs {
 };
 // y[t] = bf16(sum over the token's 8 slots of obuf, in slot order)
 cudaError_t launch_finalize(const ExpertArgs& a, cudaStream_t st);
-// persistent bulk-copy streaming versions (decode: few tokens per expert)
+// persistent streaming GEMVs (few tokens per expert): register dequant + warp MMA
 cudaError_t launch_gate_up_stream(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_down_stream(const ExpertArgs& a, cudaStream_t st);
 // tcgen05 grouped GEMMs with the dequantised weights in tensor memory;
@@ -77,6 +78,14 @@ cudaError_t launch_down_stream(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_moe_gate_up(const ExpertArgs& a, int nt, cudaStream_t st);
 cudaError_t launch_moe_down(const ExpertArgs& a, int nt, cudaStream_t st);
+
+// 2-D TMA tensor map: `inner` elements per row, `outer` rows, `pitch` bytes
+// between rows, box of box_inner x box_outer; false if the driver refuses it.
+bool encode_tma_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t pitch, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+// 3-D TMA tensor map: dims innermost first, pitch[i] = bytes between steps of dim i+1.
+bool encode_tma_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const uint64_t (&dims)[3],
+                   const uint64_t (&pitch)[2], const uint32_t (&box)[3], CUtensorMapSwizzle sw);
 
 cudaError_t launch_residual_rmsnorm(float* res, const uint16_t* y, uint16_t* x_out, int T, int H,
                                     float eps, cudaStream_t st);

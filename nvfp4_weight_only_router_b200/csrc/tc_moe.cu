@@ -437,35 +437,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* q = nullptr;
-    cudaDriverEntryPointQueryResult r;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
-        r == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(q);
-  }
-  return fn;
-}
-
-// 2-D map: inner extent `inner` elements, `outer` rows, row pitch in bytes.
-bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-               uint64_t pitch, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {pitch};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int KIND, int NT>
 cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
   static int configured_dev = -1;
@@ -482,12 +453,12 @@ cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
   CUtensorMap tm_x, tm_w;
   bool ok;
   if (KIND == kGateUp) {
-    ok = encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.xs, kH, S, kH * 2, kBK, NT, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.gu_q, kGuRowBytes, (uint64_t)kE * 2 * kI, kGuRowBytes, 32,
+    ok = encode_tma_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.xs, kH, S, kH * 2, kBK, NT, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         encode_tma_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.gu_q, kGuRowBytes, (uint64_t)kE * 2 * kI, kGuRowBytes, 32,
                    64, CU_TENSOR_MAP_SWIZZLE_NONE);
   } else {
-    ok = encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.h, kI, S, kI * 2, kBK, NT, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.dn_q, kDnRowBytes, (uint64_t)kE * kH, kDnRowBytes, 32, 64,
+    ok = encode_tma_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a.h, kI, S, kI * 2, kBK, NT, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         encode_tma_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.dn_q, kDnRowBytes, (uint64_t)kE * kH, kDnRowBytes, 32, 64,
                    CU_TENSOR_MAP_SWIZZLE_NONE);
   }
   if (!ok) return cudaErrorInvalidValue;

@@ -25,7 +25,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported(capi):
     names = header_functions()
-    assert len(names) == 14
+    assert len(names) == 15
     for n in names:
         assert hasattr(capi.lib, n), n
         assert n in capi.SIGNATURES, n
@@ -114,3 +114,8 @@ def test_residual_validation(capi):
     assert c.moe_residual_rmsnorm(None, None, P, 1, 2816, 1e-6, None) == c.NVFP4_ERR_INVALID_ARG
     assert c.moe_residual_rmsnorm(P, None, P, 1, 2817, 1e-6, None) == c.NVFP4_ERR_INVALID_ARG
     assert c.moe_residual_rmsnorm(P + 4, None, P, 1, 2816, 1e-6, None) == c.NVFP4_ERR_ALIGNMENT
+
+
+def test_last_cuda_error_is_a_string_before_any_failure(capi):
+    # no call of this thread has failed yet: the runtime's text for success
+    assert capi.lib.nvfp4_last_cuda_error().decode() == "no error"
