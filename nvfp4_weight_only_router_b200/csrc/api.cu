@@ -82,7 +82,7 @@ int stream_max_tokens() {
 struct FwdLayout {
   Region meta;
   RouteLayout route;
-  Region ids, wts, chunk_count, chunk_base, local_rank, sorted, pos, x16, xs, h, obuf;
+  Region ids, wts, chunk_count, chunk_base, local_rank, sorted, pos, xs, h, obuf;
   int S = 0, nchunks = 0;
   size_t total = 0;
 };
@@ -103,7 +103,6 @@ FwdLayout fwd_layout(int T) {
   L.local_rank = al.take(sizeof(int) * L.S);
   L.sorted = al.take(sizeof(int) * L.S);
   L.pos = al.take(sizeof(int) * L.S);
-  L.x16 = al.take(sizeof(__half) * (size_t)T * kH);
   L.xs = al.take(sizeof(__half) * (size_t)L.S * kH);
   L.h = al.take(sizeof(__half) * (size_t)L.S * kI);
   // per-slot outputs, summed in slot order by the combine: deterministic
@@ -152,7 +151,7 @@ nvfp4_status check_experts(const moe_experts* x) {
 }
 
 RouteArgs make_route_args(const void* x, int T, const moe_router* r, const RouteLayout& L, void* ws,
-                          int32_t* ids, float* wts, __half* x16, int* status) {
+                          int32_t* ids, float* wts, int* status) {
   RouteArgs a;
   a.x = static_cast<const uint16_t*>(x);
   a.proj = static_cast<const uint16_t*>(r->proj);
@@ -168,7 +167,6 @@ RouteArgs make_route_args(const void* x, int T, const moe_router* r, const Route
   a.tile_counter = at<int>(ws, L.counters);
   a.ids = ids;
   a.wts = wts;
-  a.x16 = x16;
   a.meta = nullptr;
   a.sorted_slot = nullptr;
   a.slot_pos = nullptr;
@@ -256,7 +254,7 @@ nvfp4_status moe_route(const void* x, int32_t T, const moe_router* r, int32_t* i
   cudaStream_t s = as_stream(stream);
   cudaError_t e = cudaMemsetAsync(at<int>(ws, L.counters), 0, L.counters.bytes, s);
   if (e != cudaSuccess) return cuda_fail(e);
-  RouteArgs a = make_route_args(x, T, r, L, ws, ids, w, nullptr, device_status_ptr());
+  RouteArgs a = make_route_args(x, T, r, L, ws, ids, w, device_status_ptr());
   return cuda_status(launch_route(a, s));
 }
 
@@ -317,8 +315,7 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
 
   int32_t* ids = at<int32_t>(ws, L.ids);
   float* wts = at<float>(ws, L.wts);
-  __half* x16 = at<__half>(ws, L.x16);
-  RouteArgs ra = make_route_args(x, T, r, L.route, ws, ids, wts, x16, status);
+  RouteArgs ra = make_route_args(x, T, r, L.route, ws, ids, wts, status);
   const bool fused_permute = L.S <= kFusedPermuteMaxSlots;
   if (fused_permute) {
     ra.meta = at<int>(ws, L.meta);
@@ -348,7 +345,7 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   xa.dn_q = ex->down_q;
   xa.dn_s = ex->down_s;
   xa.dn_g = ex->down_g;
-  xa.x16 = x16;
+  xa.x = static_cast<const uint16_t*>(x);
   xa.meta = pa.meta;
   xa.sorted_slot = pa.sorted_slot;
   xa.slot_pos = pa.slot_pos;

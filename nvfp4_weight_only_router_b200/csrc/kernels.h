@@ -26,7 +26,6 @@ struct RouteArgs {
   int* tile_counter;      // [ceil(T/16)], zero on entry, left zero
   int32_t* ids;           // [T, 8]
   float* wts;             // [T, 8]
-  __half* x16;            // optional f16 copy of x [T, H]
   // optional fused permutation (T*8 <= 1024): meta (route counter zero on
   // entry), sorted_slot [T*8], slot_pos [T*8]; meta == null -> not fused
   int* meta;
@@ -56,7 +55,7 @@ struct ExpertArgs {
   const uint8_t* dn_q;
   const uint8_t* dn_s;
   const float* dn_g;
-  const __half* x16;        // [T, H]
+  const uint16_t* x;        // bf16 [T, H] (the layer input)
   __half* xs;               // [S, H] activations in expert-sorted slot order
   const int* meta;
   const int* sorted_slot;   // [S]

@@ -24,7 +24,7 @@
 // Within a 128-element K segment, lane quad q holds elements [32q, 32q+32);
 // MMA step j takes elements 32q+4j+{0,1} as the fragment's low k-pair and
 // 32q+4j+{2,3} as its high k-pair, for both operands.
-#include "common.cuh"
+#include "tc_common.cuh"
 #include "kernels.h"
 
 namespace nvfp4moe {
@@ -221,7 +221,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   const uint16_t* x1 = a.x + (size_t)(v1 ? t1 : 0) * a.H + 32 * q;
   const uint16_t* prow = a.proj + (size_t)(e_base + g) * a.H + 32 * q;
   const bool do_ss = ngroup == 0;
-  const bool do_x16 = a.x16 != nullptr && eg == 0 && ngroup == 0;
 
   float acc[NTW][4];
 #pragma unroll
@@ -257,23 +256,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
           ss1 = __fmaf_rn(xb0, xb0, ss1);
           ss1 = __fmaf_rn(xb1, xb1, ss1);
         }
-      }
-      if (do_x16) {
-        // f16 copy of x for the expert GEMMs (saturating)
-        uint32_t o0[4], o1[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          o0[w] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(xaw[w] & 0xFFFFu)),
-                             f32_to_f16_sat(bf16_bits_to_f32(xaw[w] >> 16)));
-          o1[w] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(xbw[w] & 0xFFFFu)),
-                             f32_to_f16_sat(bf16_bits_to_f32(xbw[w] >> 16)));
-        }
-        if (v0)
-          *reinterpret_cast<uint4*>(a.x16 + (size_t)t0 * a.H + 32 * q + k) =
-              make_uint4(o0[0], o0[1], o0[2], o0[3]);
-        if (v1)
-          *reinterpret_cast<uint4*>(a.x16 + (size_t)t1 * a.H + 32 * q + k) =
-              make_uint4(o1[0], o1[1], o1[2], o1[3]);
       }
       const uint32_t Ah0[4] = {hi_a[0], hi_b[0], hi_a[1], hi_b[1]};
       const uint32_t Al0[4] = {lo_a[0], lo_b[0], lo_a[1], lo_b[1]};
@@ -456,20 +438,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_staged_kernel(RouteArgs a
           ss1 = __fmaf_rn(xb0, xb0, ss1);
           ss1 = __fmaf_rn(xb1, xb1, ss1);
         }
-        if (a.x16 != nullptr && eg == 0) {
-          uint32_t o0[4], o1[4];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            o0[w] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(xaw[w] & 0xFFFFu)),
-                               f32_to_f16_sat(bf16_bits_to_f32(xaw[w] >> 16)));
-            o1[w] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(xbw[w] & 0xFFFFu)),
-                               f32_to_f16_sat(bf16_bits_to_f32(xbw[w] >> 16)));
-          }
-          if (v0)
-            *reinterpret_cast<uint4*>(a.x16 + (size_t)t0 * a.H + k0 + k) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-          if (v1)
-            *reinterpret_cast<uint4*>(a.x16 + (size_t)t1 * a.H + k0 + k) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-        }
         const uint32_t Ah0[4] = {hi_a[0], hi_b[0], hi_a[1], hi_b[1]};
         const uint32_t Al0[4] = {lo_a[0], lo_b[0], lo_a[1], lo_b[1]};
         const uint32_t Ah1[4] = {hi_a[2], hi_b[2], hi_a[3], hi_b[3]};
@@ -544,9 +512,289 @@ __global__ void __launch_bounds__(kRouteThreads) route_staged_kernel(RouteArgs a
   block_permute_small(a);
 }
 
+// ------------------------------------------------------------------------
+// Cluster router.  A cluster of H/256 CTAs (11 for H = 2816) owns TOK tokens;
+// CTA r owns the K slice [256 r, 256 r + 256) for all 128 experts, so the
+// exact hi/lo split of x * scale is computed once per element.  Each CTA
+// brings its proj slice (128 x 256 bf16, four 128B-swizzled TMA boxes) and
+// its x slice (TOK x 256) into shared memory, splits x * scale into hi/lo
+// bf16 tiles, runs the two bf16 MMAs per k-step and keeps its partial logits
+// (TOK x 128 fp32) and partial sums of squares in shared memory.  After a
+// cluster barrier each CTA finishes some of the tokens, reading the partials
+// of all CTAs of the cluster in rank order (distributed shared memory, so
+// the sum has a fixed order), then softmax / top-8.  A second cluster barrier
+// keeps every CTA's shared memory alive until all reads are done.
+constexpr int kRcK = 256;  // K per CTA
+constexpr int kRcMaxRanks = 16;  // largest cluster (hidden size 4096)
+constexpr int kRcMinRanks = 8;   // smallest cluster (hidden size 2048): at most TOK / 8 tokens per CTA
+
+template <int TOK>
+struct RcSmem {
+  uint8_t proj[4][kE * 128];     // 4 K blocks of 64, rows = experts, 128B swizzle
+  uint8_t x[4][TOK * 128];       // 4 K blocks of 64, rows = tokens, 128B swizzle
+  uint16_t hi[TOK][kRcK];        // x * scale split, 16-byte chunks XOR (token & 7)
+  uint16_t lo[TOK][kRcK];
+  // partial logits and sums of squares pushed here by every CTA of the
+  // cluster for the tokens this CTA finishes (token j -> CTA j % nr, slot j / nr)
+  float red[(TOK + kRcMinRanks - 1) / kRcMinRanks][kRcMaxRanks][kE];
+  float red_ss[(TOK + kRcMinRanks - 1) / kRcMinRanks][kRcMaxRanks];
+  uint16_t scale[kRcK];
+  uint64_t bar;
+  int abort_flag;
+  int last;
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_shared(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a0, float a1) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a0), "f"(a1) : "memory");
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float a0) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a0) : "memory");
+}
+__device__ __forceinline__ uint32_t lds_u32(const void* p) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void tma_load_2d_rc(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// byte offset of element k (0..255) of row r in a hi/lo tile
+__device__ __forceinline__ uint32_t split_off(int r, int k) {
+  return (uint32_t)(r * (kRcK * 2) + ((((k >> 3) ^ (r & 7)) << 4) | ((k & 7) << 1)));
+}
+// byte offset of element k (0..63) of row r in one 128B-swizzled K block
+__device__ __forceinline__ uint32_t sw_off(int r, int k) {
+  return (uint32_t)(r * 128 + ((((k >> 3) ^ (r & 7)) << 4) | ((k & 7) << 1)));
+}
+
+template <int TOK>
+__global__ void __launch_bounds__(kRouteThreads, 1)
+    route_cluster_kernel(const __grid_constant__ CUtensorMap tm_proj, const __grid_constant__ CUtensorMap tm_x,
+                         RouteArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  RcSmem<TOK>& sm = *reinterpret_cast<RcSmem<TOK>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+  const int r = (int)cluster_ctarank(), nr = a.H / kRcK;
+  const int tok0 = blockIdx.y * TOK;
+  const int k0 = r * kRcK;
+
+  if (tid == 0) {
+    mbar_init(&sm.bar, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&sm.bar, 4 * kE * 128 + 4 * TOK * 128 + kRcK * 2);
+    for (int b = 0; b < 4; ++b) {
+      tma_load_2d_rc(smem_u32(sm.proj[b]), &tm_proj, k0 + 64 * b, 0, &sm.bar);
+      tma_load_2d_rc(smem_u32(sm.x[b]), &tm_x, k0 + 64 * b, tok0, &sm.bar);  // rows past T read as zero
+    }
+    bulk_g2s(sm.scale, a.scale + k0, kRcK * 2, &sm.bar);
+    if (!mbar_wait_bounded(&sm.bar, 0)) {
+      record_status(a.status, kStatusTimeout);
+      sm.abort_flag = 1;
+    }
+  }
+  __syncthreads();
+  const bool ok = sm.abort_flag == 0;
+
+  float acc[TOK / 16][2][4];
+#pragma unroll
+  for (int m = 0; m < TOK / 16; ++m)
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
+
+  if (ok) {
+    // split: thread k = tid of the slice, every token of the tile
+    const int k = tid, b = k >> 6, kk = k & 63;
+    const float s = bf16_bits_to_f32(sm.scale[k]);
+#pragma unroll 4
+    for (int i = 0; i < TOK; ++i) {
+      const float xv = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(sm.x[b] + sw_off(i, kk)));
+      const float pv = __fmul_rn(xv, s);
+      const __nv_bfloat16 h = __float2bfloat16_rn(pv);
+      const __nv_bfloat16 l = __float2bfloat16_rn(pv - __bfloat162float(h));
+      *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(sm.hi) + split_off(i, k)) = h;
+      *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(sm.lo) + split_off(i, k)) = l;
+    }
+    // sum of squares of x over the slice: warp w takes tokens w, w + 8, ...;
+    // lane l sums k = 8l .. 8l + 7, then a butterfly over the warp
+    for (int i = warp; i < TOK; i += kRouteThreads / 32) {
+      float q2 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int kk2 = 8 * lane + c;
+        const float xv = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(sm.x[kk2 >> 6] + sw_off(i, kk2 & 63)));
+        q2 = __fmaf_rn(xv, xv, q2);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) q2 += __shfl_xor_sync(0xffffffffu, q2, o);
+      if (lane == 0) st_cluster_f32(map_shared(&sm.red_ss[i / nr][r], (uint32_t)(i % nr)), q2);
+    }
+  }
+  __syncthreads();
+  if (ok) {
+    // MMAs: warp w owns experts [16w, 16w + 16) = two n-tiles, every m-tile;
+    // even and odd k-steps accumulate separately (shorter dependency chains)
+    float acc2[TOK / 16][2][4];
+#pragma unroll
+    for (int m = 0; m < TOK / 16; ++m)
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc2[m][n][i] = 0.f;
+#pragma unroll 2
+    for (int ks = 0; ks < kRcK / 16; ++ks) {
+      const int kb = ks * 16 + 2 * t4;  // this lane's low k-pair of the step
+      uint32_t bfr[2][2];
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const int e = 16 * warp + 8 * n + g;
+        const uint8_t* pb = sm.proj[kb >> 6];
+        bfr[n][0] = lds_u32(pb + sw_off(e, kb & 63));
+        bfr[n][1] = lds_u32(pb + sw_off(e, (kb + 8) & 63));
+      }
+#pragma unroll
+      for (int m = 0; m < TOK / 16; ++m) {
+        const int r0 = 16 * m + g;
+        const uint8_t* H = reinterpret_cast<const uint8_t*>(sm.hi);
+        const uint8_t* L = reinterpret_cast<const uint8_t*>(sm.lo);
+        const uint32_t ah[4] = {lds_u32(H + split_off(r0, kb)), lds_u32(H + split_off(r0 + 8, kb)),
+                                lds_u32(H + split_off(r0, kb + 8)), lds_u32(H + split_off(r0 + 8, kb + 8))};
+        const uint32_t al[4] = {lds_u32(L + split_off(r0, kb)), lds_u32(L + split_off(r0 + 8, kb)),
+                                lds_u32(L + split_off(r0, kb + 8)), lds_u32(L + split_off(r0 + 8, kb + 8))};
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          float (&d)[4] = (ks & 1) ? acc2[m][n] : acc[m][n];
+          mma_bf16_16816(d, ah, bfr[n][0], bfr[n][1]);
+          mma_bf16_16816(d, al, bfr[n][0], bfr[n][1]);
+        }
+      }
+    }
+    // push the partial logits to the CTA that finishes each token
+#pragma unroll
+    for (int m = 0; m < TOK / 16; ++m)
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const int e = 16 * warp + 8 * n + 2 * t4;
+#pragma unroll
+        for (int hrow = 0; hrow < 2; ++hrow) {
+          const int j = 16 * m + g + 8 * hrow;
+          st_cluster_f32x2(map_shared(&sm.red[j / nr][r][e], (uint32_t)(j % nr)),
+                           acc[m][n][2 * hrow] + acc2[m][n][2 * hrow],
+                           acc[m][n][2 * hrow + 1] + acc2[m][n][2 * hrow + 1]);
+        }
+      }
+  }
+  __syncthreads();
+  cluster_sync_all();  // every CTA's partials have landed at their owners
+
+  // finish: token j of the tile is done by CTA j % nr (slot j / nr), one
+  // warp per slot; partials summed in rank order
+  for (int sl = warp; sl * nr + r < TOK; sl += kRouteThreads / 32) {
+    const int j = sl * nr + r, t = tok0 + j;
+    if (t >= a.T) break;
+    float lg[4] = {0.f, 0.f, 0.f, 0.f}, ssum = 0.f;
+    for (int rr = 0; rr < nr; ++rr) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lg[i] += sm.red[sl][rr][lane + 32 * i];
+      ssum += sm.red_ss[sl][rr];
+    }
+    const float f = (1.0f / sqrtf(ssum / (float)a.H + a.eps)) * a.inv_sqrt_h;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) lg[i] = lg[i] * f + (a.bias ? a.bias[lane + 32 * i] : 0.f);
+    finish_token(a, t, lg);
+  }
+  __syncthreads();
+  cluster_sync_all();  // no CTA exits while peers may still store into it
+  if (!ok && tid == 0) mbar_wait_bounded(&sm.bar, 0, kAbortDrainNs);  // copies of a failed wait land first
+
+  if (a.meta == nullptr) return;
+  // few tokens: the last CTA to finish groups the slots by expert
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int prev = atomicAdd(a.meta + kMetaRouteCounter, 1);
+    sm.last = (prev == (int)(gridDim.x * gridDim.y) - 1);
+    if (sm.last) a.meta[kMetaRouteCounter] = 0;
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  block_permute_small(a);
+}
+
+template <int TOK>
+cudaError_t launch_route_cluster(const RouteArgs& a, cudaStream_t st) {
+  static int configured_dev = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const int smem = (int)sizeof(RcSmem<TOK>) + 1024;  // + alignment slack
+  if (configured_dev != dev) {
+    err = cudaFuncSetAttribute(route_cluster_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(route_cluster_kernel<TOK>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+    configured_dev = dev;
+  }
+  const int nr = a.H / kRcK;
+  CUtensorMap tm_proj, tm_x;
+  if (!encode_tma_2d(&tm_proj, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.proj, (uint64_t)a.H, kE, (uint64_t)a.H * 2, 64, kE,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tma_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.H, (uint64_t)a.T, (uint64_t)a.H * 2, 64,
+                     TOK, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nr, (a.T + TOK - 1) / TOK, 1);
+  cfg.blockDim = dim3(kRouteThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nr;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, route_cluster_kernel<TOK>, tm_proj, tm_x, a);
+}
+
+static_assert(sizeof(RcSmem<16>) + 1024 + 8192 <= 232448, "shared memory budget of the cluster router");
+
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
+  // few tokens and hidden sizes of 8 to 16 slices of 256: one cluster per 16 tokens
+  if (a.few_tokens && a.H % kRcK == 0 && a.H / kRcK >= kRcMinRanks && a.H / kRcK <= kRcMaxRanks)
+    return launch_route_cluster<16>(a, st);
   if (a.few_tokens) {
     static int configured_dev = -1;
     int dev = 0;

@@ -18,10 +18,12 @@
 // (A row 2r = gate r, 2r+1 = up r), so the GELU gate of a hidden unit is a
 // shuffle between adjacent lanes.
 //
-// Warp roles (16 warps): 0 TMA producer (activation box, packed-code boxes,
-// the tile's E4M3 scales by a bulk copy), 1 MMA issuer (one thread),
-// 4-7 epilogue (tensor memory -> registers -> global), 8-15 dequantisation
-// (warp w owns tensor-memory lanes 32(w%4).. and K half (w-8)/4).
+// Warp roles (16 warps): 0 TMA producer (activation box, packed-code boxes),
+// 1-3 MMA issuers (one thread each; from 64 tokens on two or three split the
+// tile's tokens), 4-7 epilogue (tensor memory -> registers -> global), 8-15
+// dequantisation (warp w owns tensor-memory lanes 32(w%4).. and K half
+// (w-8)/4; it reads its row's e4m3 scales from global memory three chunks
+// ahead, so the shared memory goes to a deeper load ring).
 // Every wait is bounded in wall time; a wait that gives up records a timeout
 // status, and the CTA drains its copies and MMAs, frees its tensor memory and
 // exits.
@@ -46,21 +48,27 @@ struct Cfg {
   static constexpr int NJ = KIND == kGateUp ? (2 * kI) / kRows : kH / kRows;  // 11 or 22 row tiles
   static constexpr int KC = (KIND == kGateUp ? kH : kI) / kBK;               // 44 or 11 chunks
   static constexpr int SROW = KIND == kGateUp ? kGuScaleRow : kDnScaleRow;   // scale bytes per row
-  static constexpr int SC_BYTES = kRows * SROW;                             // scales of a tile
   static constexpr int X_BYTES = NT * 128;
   static constexpr int CODE_BYTES = kRows * 32;
-  // epilogue staging per warp: gate_up h values (NT tokens x 16 units, f16),
-  // down one 16-token chunk of 32 rows (fp32)
-  static constexpr int STAGE_BYTES = KIND == kGateUp ? NT * 32 : 16 * 32 * 4;
+  // epilogue staging per warp: gate_up h values (NT tokens x 16 units, f16);
+  // down stores straight from registers
+  static constexpr int STAGE_BYTES = KIND == kGateUp ? NT * 32 : 16;
   // load stages: as many as fit next to the scale buffers and the staging
-  static constexpr int NS_RAW = (206 * 1024 - 2 * SC_BYTES - 4 * STAGE_BYTES) / (X_BYTES + CODE_BYTES);
+  static constexpr int NS_RAW = (222 * 1024 - 4 * STAGE_BYTES) / (X_BYTES + CODE_BYTES);
   static constexpr int NS = NS_RAW > 24 ? 24 : NS_RAW;
   static constexpr int NA = 4;                                             // A stages (32 columns each)
+  static_assert(NA <= NS, "an A stage is released through the empty barrier of its chunk's load stage");
   // independent accumulators per tile: small-N MMAs into one accumulator
   // would wait on each other, so the K sub-steps rotate over NACC of them
   static constexpr int NACC = NT <= 16 ? 4 : (NT <= 64 ? 2 : 1);
   static constexpr int ND = (2 * NACC * NT + NA * 32 <= kTmemCols) ? 2 : 1; // accumulator buffers
   static constexpr int A_COL0 = ND * NACC * NT;                           // first A-stage column
+  // MMA-issuing warps: one thread issues a tcgen05.mma only every ~110
+  // cycles, well below the tensor core's rate, so from 64 tokens on two or
+  // three warps split the tile's tokens (N), each with its own share of the
+  // accumulator columns and of the activation rows
+  static constexpr int NI = NT >= 192 ? 3 : (NT >= 64 ? 2 : 1);
+  static constexpr int NH = NT / NI;                                      // MMA N per issuer
   static_assert(A_COL0 + NA * 32 <= kTmemCols, "tensor memory budget");
 };
 
@@ -69,17 +77,17 @@ struct alignas(1024) MoeSmem {
   using C = Cfg<KIND, NT>;
   uint8_t x[C::NS][C::X_BYTES];          // B tiles (SW128, 1024-aligned since X_BYTES % 1024 == 0)
   uint8_t code[C::NS][C::CODE_BYTES];    // packed codes: 128 rows x 32 bytes
-  uint8_t sc[2][C::SC_BYTES];            // E4M3 scales of a tile (rows in tile-row order)
   uint8_t stage[4][C::STAGE_BYTES];      // epilogue staging, one per epilogue warp
+  // empty[s]: the MMAs of the chunk in stage s completed, so both its shared
+  // memory stage and its tensor-memory A stage (NA <= NS) are free again
   uint64_t full[C::NS], empty[C::NS];
-  uint64_t a_full[C::NA], a_empty[C::NA];
-  uint64_t sc_full[2], sc_empty[2];
+  uint64_t a_full[C::NA];
   uint64_t d_full[2], d_empty[2];
   uint64_t fin;
   uint32_t taddr;
   int mt_prefix[kE + 1];
   int abort_flag;
-  int issued_chunks, issued_tiles;       // producer progress (for draining after an abort)
+  int issued_chunks;                     // producer progress (for draining after an abort)
   float wslot[4][NT];                    // down: routing weight x G_d per token (one copy per epilogue warp)
 };
 
@@ -185,22 +193,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       for (int s = 0; s < C::NS; ++s) {
         mbar_init(&sm.full[s], 1);
-        mbar_init(&sm.empty[s], 1);
+        mbar_init(&sm.empty[s], C::NI);
       }
       for (int a = 0; a < C::NA; ++a) {
         mbar_init(&sm.a_full[a], 8);    // one arrival per dequant warp
-        mbar_init(&sm.a_empty[a], 1);
       }
       for (int b = 0; b < 2; ++b) {
-        mbar_init(&sm.sc_full[b], 1);
-        mbar_init(&sm.sc_empty[b], 8);
-        mbar_init(&sm.d_full[b], 1);
+        mbar_init(&sm.d_full[b], C::NI);
         mbar_init(&sm.d_empty[b], 4);   // one arrival per epilogue warp
       }
-      mbar_init(&sm.fin, 1);
+      mbar_init(&sm.fin, C::NI);
       sm.abort_flag = 0;
       sm.issued_chunks = 0;
-      sm.issued_tiles = 0;
       fence_mbar_init();
     }
   }
@@ -217,25 +221,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpProd) {
     // -------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const uint8_t* sc_src = KIND == kGateUp ? p.gu_s : p.dn_s;
-      uint32_t kiter = 0, titer = 0;
+      uint32_t kiter = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++titer) {
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         const TileInfo ti = decode_tile<KIND, NT>(sm, p.meta, t);
         const int xrow = ti.off + ti.i * NT;
-        // the tile's scales: gate_up = two runs of 64 rows (gate, up), down = one run of 128
-        const int sb = titer & 1, suse = titer >> 1;
-        if (suse > 0 && !wait_or_abort(sm, &sm.sc_empty[sb], (suse - 1) & 1, p.status)) break;
-        mbar_arrive_expect_tx(&sm.sc_full[sb], C::SC_BYTES);
-        if (KIND == kGateUp) {
-          const int g0 = tile_row<KIND>(ti.e, ti.j, 0), u0 = tile_row<KIND>(ti.e, ti.j, 1);
-          bulk_g2s_u32(smem_u32(sm.sc[sb]), sc_src + (size_t)g0 * C::SROW, 64 * C::SROW, &sm.sc_full[sb]);
-          bulk_g2s_u32(smem_u32(sm.sc[sb]) + 64 * C::SROW, sc_src + (size_t)u0 * C::SROW, 64 * C::SROW,
-                       &sm.sc_full[sb]);
-        } else {
-          const int r0 = tile_row<KIND>(ti.e, ti.j, 0);
-          bulk_g2s_u32(smem_u32(sm.sc[sb]), sc_src + (size_t)r0 * C::SROW, C::SC_BYTES, &sm.sc_full[sb]);
-        }
         for (int kc = 0; kc < C::KC; ++kc, ++kiter) {
           const int s = kiter % C::NS, use = kiter / C::NS;
           if (use > 0 && !wait_or_abort(sm, &sm.empty[s], (use - 1) & 1, p.status)) { ok = false; break; }
@@ -248,7 +238,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(smem_u32(sm.code[s]) + 64 * 32, &tm_w, kc * 32, rb, &sm.full[s]);
           sm.issued_chunks = kiter + 1;
         }
-        sm.issued_tiles = titer + 1;
       }
     }
   } else if (warp >= kWarpDeq0) {
@@ -257,19 +246,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int L = quarter * 32 + lane;  // tensor-memory lane = A row
     // code / scale row in shared memory: gate_up stores gate rows 0..63 then up rows 64..127
     const int crow = KIND == kGateUp ? ((L & 1) * 64 + (L >> 1)) : L;
-    uint32_t kiter = 0, titer = 0;
+    // this lane's e4m3 scale pair of each chunk, read from global memory
+    // three chunks ahead of its use (the walk crosses tile boundaries)
+    const uint8_t* sc_src = KIND == kGateUp ? p.gu_s : p.dn_s;
+    int pt = blockIdx.x, pkc = 0;
+    const uint8_t* prow = nullptr;
+    auto prow_of = [&](int t) -> const uint8_t* {
+      const TileInfo ti = decode_tile<KIND, NT>(sm, p.meta, t);
+      return sc_src + (size_t)tile_row<KIND>(ti.e, ti.j, L) * C::SROW + khalf * 2;
+    };
+    if (pt < n_tiles) prow = prow_of(pt);
+    auto next_scale = [&]() -> uint16_t {
+      if (pt >= n_tiles) return 0;
+      const uint16_t v = ldg_nc_u16(prow + pkc * 4);
+      if (++pkc == C::KC) {
+        pkc = 0;
+        pt += gridDim.x;
+        if (pt < n_tiles) prow = prow_of(pt);
+      }
+      return v;
+    };
+    uint16_t sq0 = next_scale(), sq1 = next_scale(), sq2 = next_scale();
+    uint32_t kiter = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++titer) {
-      const int sb = titer & 1, suse = titer >> 1;
-      if (!wait_or_abort(sm, &sm.sc_full[sb], suse & 1, p.status)) break;
-      const uint8_t* scrow = sm.sc[sb] + crow * C::SROW;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
       for (int kc = 0; kc < C::KC; ++kc, ++kiter) {
         const int s = kiter % C::NS, use = kiter / C::NS;
         const int a = kiter % C::NA, ause = kiter / C::NA;
+        const uint16_t sq = sq0;
+        sq0 = sq1;
+        sq1 = sq2;
+        sq2 = next_scale();
         if (!wait_or_abort(sm, &sm.full[s], use & 1, p.status)) { ok = false; break; }
-        if (ause > 0 && !wait_or_abort(sm, &sm.a_empty[a], (ause - 1) & 1, p.status)) { ok = false; break; }
+        // A stage a was last used by chunk kiter - NA (its MMAs signal empty[] of that chunk's stage)
+        if (ause > 0 && !wait_or_abort(sm, &sm.empty[(kiter - C::NA) % C::NS], ((kiter - C::NA) / C::NS) & 1, p.status)) {
+          ok = false;
+          break;
+        }
         const uint4 w = lds_v4(sm.code[s] + crow * 32 + khalf * 16);   // 32 K of this row
-        const uint32_t s2 = e4m3x2_to_f16x2(lds_u16(scrow + kc * 4 + khalf * 2));
+        const uint32_t s2 = e4m3x2_to_f16x2(sq);
         const uint32_t slo = bcast_lo(s2), shi = bcast_hi(s2);
         const uint32_t words[4] = {w.x, w.y, w.z, w.w};
         uint32_t v[16];
@@ -287,20 +302,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.a_full[a]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.sc_empty[sb]);
     }
-  } else if (warp == kWarpMma) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp >= kWarpMma && warp < kWarpMma + C::NI) {
+    // ---------------------------------------------------------- MMA issuers
     if (lane == 0) {
-      const uint32_t idesc = make_idesc_f16(kRows, NT);
+      const int hh = warp - kWarpMma;  // token share of this issuer
       uint32_t kiter = 0, titer = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++titer) {
         const int db = titer % C::ND, duse = titer / C::ND;
+        // only the columns of the tile's valid tokens (rounded up to 16): the
+        // tensor core's time grows with N, and an expert's last tile is often
+        // mostly empty; an issuer with no valid column issues nothing
+        const TileInfo ti = decode_tile<KIND, NT>(sm, p.meta, t);
+        const int mine = min(C::NH, min(NT, ti.cnt - ti.i * NT) - hh * C::NH);
+        const int nmma = mine <= 0 ? 0 : ((mine + 15) & ~15);
+        const uint32_t idesc = make_idesc_f16(kRows, nmma > 0 ? nmma : 16);
         if (duse > 0 && !wait_or_abort(sm, &sm.d_empty[db], (duse - 1) & 1, p.status)) break;
         tc_fence_after();
-        const uint32_t d = taddr + (uint32_t)(db * C::NACC * NT);
+        const uint32_t d = taddr + (uint32_t)(db * C::NACC * NT + hh * C::NH);
         for (int kc = 0; kc < C::KC; ++kc, ++kiter) {
           const int s = kiter % C::NS, use = kiter / C::NS;
           const int a = kiter % C::NA, ause = kiter / C::NA;
@@ -310,14 +330,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t bd = make_sw128_desc(smem_u32(sm.x[s]));
+          // rows hh*NH.. of the 128B-swizzled activation tile (NH*128 bytes = whole 8-row atoms)
+          const uint64_t bd = make_sw128_desc(smem_u32(sm.x[s]) + (uint32_t)(hh * C::NH * 128));
           const uint32_t a0 = taddr + (uint32_t)(C::A_COL0 + a * 32);
+          if (nmma > 0) {
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma_ts(d + (uint32_t)((kk % C::NACC) * NT), a0 + (uint32_t)(kk * 8), bd + (uint64_t)(kk * 2), idesc,
-                      kc != 0 || kk >= C::NACC);
-          tc_commit(&sm.empty[s]);
-          tc_commit(&sm.a_empty[a]);
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              tc_mma_ts(d + (uint32_t)((kk % C::NACC) * NT), a0 + (uint32_t)(kk * 8), bd + (uint64_t)(kk * 2), idesc,
+                        kc != 0 || kk >= C::NACC);
+          }
+          tc_commit(&sm.empty[s]);  // with no MMA in flight the arrival is immediate
         }
         if (!ok) break;
         tc_commit(&sm.d_full[db]);
@@ -339,8 +361,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // routing weight x G_d of each token column, in this warp's own copy
         __syncwarp();
         const float G = p.dn_g[ti.e];
-        for (int n = lane; n < NT; n += 32)
-          sm.wslot[quarter][n] = n < nvalid ? p.wts[p.sorted_slot[pos0 + n]] * G : 0.f;
+        // all slot ids first, then all weights: two memory round trips per tile
+        constexpr int PER = (NT + 31) / 32;
+        int slot[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          const int n = lane + 32 * i;
+          slot[i] = n < nvalid ? __ldg(p.sorted_slot + pos0 + n) : -1;
+        }
+        float wv[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) wv[i] = slot[i] >= 0 ? __ldg(p.wts + slot[i]) : 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+          if (lane + 32 * i < NT) sm.wslot[quarter][lane + 32 * i] = wv[i] * G;
         __syncwarp();
       }
       if (!wait_or_abort(sm, &sm.d_full[db], duse & 1, p.status)) break;
@@ -354,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float G = p.gu_g[ti.e];
         const bool odd = L & 1;
         const int ul = lane >> 1;  // unit within the warp's 16
-        for (int cc = 0; cc < NT / 16; ++cc) {
+        for (int cc = 0; cc * 16 < nvalid; ++cc) {
           float v[16];
           tmem_ld16(trow + cc * 16, v);
 #pragma unroll
@@ -385,32 +419,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       } else {
-        // 16-token chunks: rows of this warp x tokens -> staging [token][32 rows]
-        // -> one 16-byte store per 4 rows of a token
-        const int row0 = ti.j * kRows + quarter * 32;
-        float* st = reinterpret_cast<float*>(stg);
-        for (int cc = 0; cc < NT / 16; ++cc) {
-          float v[16];
-          tmem_ld16(trow + cc * 16, v);
+        // lane = output row; per token one 4-byte store per lane, i.e. 128
+        // contiguous bytes per warp store; only the tile's valid tokens
+        const int row = ti.j * kRows + quarter * 32 + lane;
+        constexpr int CW = NT % 32 == 0 ? 32 : 16;  // tokens per tensor-memory load
+        for (int cc = 0; cc * CW < nvalid; ++cc) {
+          float v[CW];
+          if constexpr (CW == 32) tmem_ld32(trow + cc * CW, v); else tmem_ld16(trow + cc * CW, v);
 #pragma unroll
           for (int acc = 1; acc < C::NACC; ++acc) {
-            float w[16];
-            tmem_ld16(trow + acc * NT + cc * 16, w);
+            float w[CW];
+            if constexpr (CW == 32) tmem_ld32(trow + acc * NT + cc * CW, w); else tmem_ld16(trow + acc * NT + cc * CW, w);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] += w[k];
+            for (int k = 0; k < CW; ++k) v[k] += w[k];
           }
+          const int nmax = min(CW, nvalid - cc * CW);
 #pragma unroll
-          for (int k = 0; k < 16; ++k) st[k * 32 + lane] = v[k] * sm.wslot[quarter][cc * 16 + k];
-          __syncwarp();
-          const int nmax = min(16, nvalid - cc * 16);
-#pragma unroll
-          for (int rep4 = 0; rep4 < 4; ++rep4) {
-            const int k = rep4 * 4 + (lane >> 3), r4 = (lane & 7) * 4;
-            if (k < nmax)
-              *reinterpret_cast<float4*>(p.obuf + (size_t)(pos0 + cc * 16 + k) * kH + row0 + r4) =
-                  *reinterpret_cast<const float4*>(st + k * 32 + r4);
-          }
-          __syncwarp();
+          for (int k = 0; k < CW; ++k)
+            if (k < nmax) p.obuf[(size_t)(pos0 + cc * CW + k) * kH + row] = v[k] * sm.wslot[quarter][cc * CW + k];
         }
       }
       tc_fence_before();
@@ -427,8 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (older stages were reused, so only the last NS chunks and 2 tiles can be)
     for (int it = max(0, sm.issued_chunks - C::NS); it < sm.issued_chunks; ++it)
       mbar_wait_bounded(&sm.full[it % C::NS], (it / C::NS) & 1, kAbortDrainNs);
-    for (int it = max(0, sm.issued_tiles - 2); it < sm.issued_tiles; ++it)
-      mbar_wait_bounded(&sm.sc_full[it & 1], (it >> 1) & 1, kAbortDrainNs);
   }
   __syncthreads();
   if (warp == kWarpMma) {
@@ -436,6 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(taddr, kTmemCols);
   }
 }
+
+static_assert(sizeof(MoeSmem<kGateUp, 192>) + 1024 <= 232448, "shared memory budget (gate_up)");
+static_assert(sizeof(MoeSmem<kDown, 192>) + 1024 <= 232448, "shared memory budget (down)");
 
 template <int KIND, int NT>
 cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
@@ -469,9 +496,10 @@ cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// x_sorted[pos] = x16[token of sorted slot pos]: the activations in expert
-// order, so that every tile of the expert GEMMs reads contiguous rows.
-__global__ void __launch_bounds__(256) gather_sorted_kernel(const __half* __restrict__ x16,
+// xs[pos] = f16(x[token of sorted slot pos]) (saturating): the activations in
+// expert order and in the f16 of the MMA operands, so that every tile of the
+// expert GEMMs reads contiguous rows.  One thread per 8 elements.
+__global__ void __launch_bounds__(256) gather_sorted_kernel(const uint16_t* __restrict__ x,
                                                             const int* __restrict__ sorted_slot,
                                                             const int* __restrict__ meta, int T,
                                                             __half* __restrict__ xs, int* status) {
@@ -485,7 +513,13 @@ __global__ void __launch_bounds__(256) gather_sorted_kernel(const __half* __rest
       record_status(status, kStatusDevice);
       tok = 0;
     }
-    reinterpret_cast<uint4*>(xs + (size_t)pos * kH)[c] = reinterpret_cast<const uint4*>(x16 + (size_t)tok * kH)[c];
+    const uint4 v = ldg_nc_v4(x + (size_t)tok * kH + 8 * c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      o[k] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(w[k] & 0xFFFFu)), f32_to_f16_sat(bf16_bits_to_f32(w[k] >> 16)));
+    reinterpret_cast<uint4*>(xs + (size_t)pos * kH)[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -495,7 +529,7 @@ cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st) {
   const int64_t n = (int64_t)a.T * kTopK * (kH / 8);
   int blocks = (int)((n + 255) / 256);
   if (blocks > 4096) blocks = 4096;
-  gather_sorted_kernel<<<blocks, 256, 0, st>>>(a.x16, a.sorted_slot, a.meta, a.T, a.xs, a.status);
+  gather_sorted_kernel<<<blocks, 256, 0, st>>>(a.x, a.sorted_slot, a.meta, a.T, a.xs, a.status);
   return cudaGetLastError();
 }
 
