@@ -273,13 +273,25 @@ def run_ours(args, wl, rank, world, local_rank):
         xs.copy_(x_pool[0])
         step_body(True)
         torch.cuda.synchronize()
+        # two graphs of the same step: a plain one for the timed steps, and one
+        # with event-record nodes between the phases for the phase breakdown
+        # (event nodes cost launch gaps, so they stay out of the headline time)
+        graph_prof = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_prof):
+            step_body(True)
+        torch.cuda.synchronize()
+        step_body(False)
+        torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            step_body(True)
+            step_body(False)
         torch.cuda.synchronize()
 
         def step(i):
             graph.replay()
+
+        def step_prof(i):
+            graph_prof.replay()
 
         def prepare(i):
             xs.copy_(x_pool[i % n_pool])
@@ -314,8 +326,22 @@ def run_ours(args, wl, rank, world, local_rank):
         torch.cuda.synchronize()
         step_ms.append(start.elapsed_time(end))
         if args.workload != "quantize":
-            phase_ms.append([events[j].elapsed_time(events[j + 1]) for j in range(5)])
             act_counts.append(int((layers[0].views(T)["counts"] > 0).sum().item()))
+    torch.cuda.synchronize()
+    # phase breakdown (and the dominant kernel's duration for the roofline):
+    # the same K steps again, each replaying the graph whose event-record
+    # nodes sit between the phases, on the launching stream
+    prof_ms = []
+    if args.workload != "quantize":
+        for k in range(args.steps):
+            flush.zero_()
+            prepare(k)
+            start.record()
+            step_prof(k)
+            end.record()
+            torch.cuda.synchronize()
+            prof_ms.append(start.elapsed_time(end))
+            phase_ms.append([events[j].elapsed_time(events[j + 1]) for j in range(5)])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -385,6 +411,7 @@ def run_ours(args, wl, rank, world, local_rank):
         extra = {
             "phase_ms_mean": dict(zip(["route", "permute", "gate_up", "down", "combine"],
                                       [float(v) for v in ph.mean(0)])),
+            "ms_per_step_with_phase_events": float(np.mean(prof_ms)),
             "active_experts_mean": float(n_act.mean()),
             # whole-step algorithmic bytes (active experts + router + x + y) per second
             "step_hbm_gbs": float(step_bytes.mean() * wl["layers"] / (ms_per_step / 1e3) / 1e9),
@@ -418,7 +445,7 @@ def run_ours(args, wl, rank, world, local_rank):
         line.update(extra)
         print(json.dumps(line), flush=True)
     if args.workload != "quantize":
-        del graph
+        del graph, graph_prof
 
 
 def main():

@@ -336,7 +336,6 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   pa.slot_pos = at<int>(ws, L.pos);
   pa.status = status;
   if (!fused_permute && (e = launch_permute(pa, s)) != cudaSuccess) return cuda_fail(e);
-  if (!mark(2)) return cuda_fail(cudaGetLastError());
 
   ExpertArgs xa;
   xa.gu_q = ex->gate_up_q;
@@ -357,7 +356,9 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   xa.max_active = L.S < kE ? L.S : kE;
   xa.status = status;
   xa.xs = at<__half>(ws, L.xs);
+  // the activations follow their slots into expert order (f16 for the MMAs)
   if ((e = launch_gather_sorted(xa, s)) != cudaSuccess) return cuda_fail(e);
+  if (!mark(2)) return cuda_fail(cudaGetLastError());
   if (T <= stream_max_tokens()) {
     // few tokens per expert: the weight stream bounds the step (streaming
     // GEMV with register dequantisation)
