@@ -82,7 +82,7 @@ int stream_max_tokens() {
 struct FwdLayout {
   Region meta;
   RouteLayout route;
-  Region ids, wts, chunk_count, chunk_base, local_rank, sorted, pos, xs, h, obuf;
+  Region ids, wts, chunk_count, sorted, pos, xs, h, obuf;
   int S = 0, nchunks = 0;
   size_t total = 0;
 };
@@ -99,8 +99,6 @@ FwdLayout fwd_layout(int T) {
   L.ids = al.take(sizeof(int) * L.S);
   L.wts = al.take(sizeof(float) * L.S);
   L.chunk_count = al.take(sizeof(int) * (size_t)L.nchunks * kE);
-  L.chunk_base = al.take(sizeof(int) * (size_t)L.nchunks * kE);
-  L.local_rank = al.take(sizeof(int) * L.S);
   L.sorted = al.take(sizeof(int) * L.S);
   L.pos = al.take(sizeof(int) * L.S);
   L.xs = al.take(sizeof(__half) * (size_t)L.S * kH);
@@ -330,8 +328,6 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   pa.nchunks = L.nchunks;
   pa.meta = at<int>(ws, L.meta);
   pa.chunk_count = at<int>(ws, L.chunk_count);
-  pa.chunk_base = at<int>(ws, L.chunk_base);
-  pa.local_rank = at<int>(ws, L.local_rank);
   pa.sorted_slot = at<int>(ws, L.sorted);
   pa.slot_pos = at<int>(ws, L.pos);
   pa.status = status;

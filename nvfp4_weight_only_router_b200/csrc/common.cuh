@@ -38,7 +38,6 @@ constexpr int kMetaCounts = 0;      // [E] tokens routed to each expert
 constexpr int kMetaOffsets = 128;   // [E+1] exclusive prefix of counts
 constexpr int kMetaAct = 260;       // [E] ids of experts with count > 0, ascending
 constexpr int kMetaNAct = 388;      // number of active experts
-constexpr int kMetaPermCounter = 392;  // arrival counter of the permute kernel
 constexpr int kMetaRouteCounter = 396; // arrival counter of the router's token tiles
 constexpr int kMetaInts = 512;
 

@@ -38,10 +38,8 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 struct PermuteArgs {
   const int32_t* ids;  // [S]
   int S, nchunks;
-  int* meta;           // kMetaInts ints (counter zero on entry, left zero)
-  int* chunk_count;    // [nchunks, 128]
-  int* chunk_base;     // [nchunks, 128]
-  int* local_rank;     // [S]
+  int* meta;           // kMetaInts ints (written: counts, offsets, active list)
+  int* chunk_count;    // [nchunks, 128] per-chunk counts (scratch)
   int* sorted_slot;    // [S]
   int* slot_pos;       // [S]
   int* status;

@@ -3,14 +3,14 @@
 // only ...").  Slots s = t*8 + j are grouped by expert id with a stable
 // counting sort, so each expert's slots stay in token order.
 //
-// Each CTA takes a chunk of 1024 slots (one per thread):
-//   phase A: within-warp ranks by __match_any_sync, per-warp per-expert
-//            counts in shared memory, a scan over the 32 warps -> each slot's
-//            rank inside its chunk and the chunk's per-expert counts;
-//   the last CTA to arrive (arrival counter) then runs
-//   phase B: per-expert prefix over chunks, exclusive scan over experts
-//            (offsets), the list of active experts;
-//   phase C: scatter: pos = offsets[e] + chunk_base[chunk][e] + local rank.
+// Two launches over chunks of 1024 slots (one per thread):
+//   count:   each CTA writes its chunk's per-expert counts;
+//   scatter: each CTA recomputes its slots' ranks inside the chunk (within-
+//            warp ranks by __match_any_sync, a scan over the 32 warps), reads
+//            the count table to get its chunk's base per expert and every
+//            expert's offset, and places its slots: pos = offset[e] +
+//            base[chunk][e] + rank.  CTA 0 also writes the counts, offsets
+//            and the active-expert list.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -42,22 +42,19 @@ __device__ __forceinline__ int warp_exclusive_scan128(int (&v)[4]) {
   return total;
 }
 
-__global__ void __launch_bounds__(kChunk) permute_kernel(PermuteArgs a) {
-  __shared__ int wcount[32][kE];
-  __shared__ int s_last;
-  __shared__ int s_off[kE + 1];
+// ranks of the chunk's slots inside the chunk: per-warp per-expert counts in
+// wcount (then their exclusive scan over warps); returns the slot's expert
+// (-1 if none or invalid) and its rank
+__device__ __forceinline__ int chunk_rank(const PermuteArgs& a, int (*wcount)[kE], int& e_out, bool write_counts) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x;
-
   for (int i = tid; i < 32 * kE; i += kChunk) (&wcount[0][0])[i] = 0;
   __syncthreads();
-
-  const int s = chunk * kChunk + tid;
+  const int s = blockIdx.x * kChunk + tid;
   int e = -1;
   if (s < a.S) {
     e = a.ids[s];
     if (e < 0 || e >= kE) {
-      record_status(a.status, kStatusDevice);
+      if (write_counts) record_status(a.status, kStatusDevice);
       e = -1;
     }
   }
@@ -72,31 +69,52 @@ __global__ void __launch_bounds__(kChunk) permute_kernel(PermuteArgs a) {
       wcount[w][tid] = run;
       run += c;
     }
-    a.chunk_count[(size_t)chunk * kE + tid] = run;
+    if (write_counts) a.chunk_count[(size_t)blockIdx.x * kE + tid] = run;
   }
   __syncthreads();
-  if (s < a.S) a.local_rank[s] = (e >= 0) ? wcount[warp][e] + rank : 0;
+  e_out = e;
+  return e >= 0 ? wcount[warp][e] + rank : 0;
+}
 
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int prev = atomicAdd(a.meta + kMetaPermCounter, 1);
-    s_last = (prev == (int)gridDim.x - 1);
-    if (s_last) a.meta[kMetaPermCounter] = 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+__global__ void __launch_bounds__(kChunk) permute_count_kernel(PermuteArgs a) {
+  __shared__ int wcount[32][kE];
+  int e;
+  chunk_rank(a, wcount, e, true);
+}
 
-  // phase B: per-expert prefix over chunks
-  if (tid < kE) {
-    int run = 0;
-    for (int c = 0; c < a.nchunks; ++c) {
-      const int v = __ldcg(a.chunk_count + (size_t)c * kE + tid);
-      a.chunk_base[(size_t)c * kE + tid] = run;
-      run += v;
+__global__ void __launch_bounds__(kChunk) permute_scatter_kernel(PermuteArgs a) {
+  __shared__ int wcount[32][kE];
+  __shared__ int part_tot[8][kE], part_base[8][kE];
+  __shared__ int s_off[kE + 1], s_base[kE];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x;
+  int e;
+  const int rank = chunk_rank(a, wcount, e, false);
+
+  // per expert: its total over all chunks and its base in this chunk (the
+  // counts of the chunks before it); thread (expert ex, part p) takes chunks
+  // c = p, p + 8, ...
+  {
+    const int ex = tid & (kE - 1), part = tid >> 7;
+    int tot = 0, base = 0;
+    for (int c = part; c < a.nchunks; c += 8) {
+      const int v = a.chunk_count[(size_t)c * kE + ex];
+      tot += v;
+      if (c < chunk) base += v;
     }
-    s_off[tid] = run;  // count of expert tid (scanned below)
+    part_tot[part][ex] = tot;
+    part_base[part][ex] = base;
+  }
+  __syncthreads();
+  if (tid < kE) {
+    int tot = 0, base = 0;
+#pragma unroll
+    for (int pt = 0; pt < 8; ++pt) {
+      tot += part_tot[pt][tid];
+      base += part_base[pt][tid];
+    }
+    s_off[tid] = tot;
+    s_base[tid] = base;
   }
   __syncthreads();
   if (warp == 0) {
@@ -105,7 +123,6 @@ __global__ void __launch_bounds__(kChunk) permute_kernel(PermuteArgs a) {
     for (int i = 0; i < 4; ++i) {
       cnt[i] = s_off[4 * lane + i];
       flag[i] = cnt[i] > 0;
-      a.meta[kMetaCounts + 4 * lane + i] = cnt[i];
     }
     int off[4] = {cnt[0], cnt[1], cnt[2], cnt[3]};
     const int total = warp_exclusive_scan128(off);
@@ -115,34 +132,40 @@ __global__ void __launch_bounds__(kChunk) permute_kernel(PermuteArgs a) {
     for (int i = 0; i < 4; ++i) {
       const int ex = 4 * lane + i;
       s_off[ex] = off[i];
-      a.meta[kMetaOffsets + ex] = off[i];
-      if (cnt[i] > 0) a.meta[kMetaAct + flag[i]] = ex;
+      if (chunk == 0) {
+        a.meta[kMetaCounts + ex] = cnt[i];
+        a.meta[kMetaOffsets + ex] = off[i];
+        if (cnt[i] > 0) a.meta[kMetaAct + flag[i]] = ex;
+      }
     }
     if (lane == 0) {
       s_off[kE] = total;
-      a.meta[kMetaOffsets + kE] = total;
-      a.meta[kMetaNAct] = nact;
+      if (chunk == 0) {
+        a.meta[kMetaOffsets + kE] = total;
+        a.meta[kMetaNAct] = nact;
+      }
     }
   }
   __syncthreads();
-
-  // phase C: scatter
-  for (int ss = tid; ss < a.S; ss += kChunk) {
-    const int ee = a.ids[ss];
-    if (ee < 0 || ee >= kE) {
-      a.slot_pos[ss] = -1;
-      continue;
+  const int s = chunk * kChunk + tid;
+  if (s < a.S) {
+    if (e < 0) {
+      a.slot_pos[s] = -1;
+    } else {
+      const int pos = s_off[e] + s_base[e] + rank;
+      a.sorted_slot[pos] = s;
+      a.slot_pos[s] = pos;
     }
-    const int pos = s_off[ee] + a.chunk_base[(size_t)(ss / kChunk) * kE + ee] + __ldcg(a.local_rank + ss);
-    a.sorted_slot[pos] = ss;
-    a.slot_pos[ss] = pos;
   }
 }
 
 }  // namespace
 
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
-  permute_kernel<<<a.nchunks, kChunk, 0, st>>>(a);
+  permute_count_kernel<<<a.nchunks, kChunk, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  permute_scatter_kernel<<<a.nchunks, kChunk, 0, st>>>(a);
   return cudaGetLastError();
 }
 

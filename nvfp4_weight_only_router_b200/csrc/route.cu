@@ -569,6 +569,15 @@ __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a0, float 
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float a0) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a0) : "memory");
 }
+// four 8x8 b16 matrices from shared memory, lane l giving the 16-byte row
+// address of row l % 8 of matrix l / 8; register i holds matrix i in the
+// warp-MMA fragment order (row l / 4, elements 2 (l % 4) and 2 (l % 4) + 1)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+      : "r"(addr)
+      : "memory");
+}
 __device__ __forceinline__ uint32_t lds_u32(const void* p) {
   uint32_t v;
   asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
@@ -632,17 +641,19 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       for (int i = 0; i < 4; ++i) acc[m][n][i] = 0.f;
 
   if (ok) {
-    // split: thread k = tid of the slice, every token of the tile
-    const int k = tid, b = k >> 6, kk = k & 63;
-    const float s = bf16_bits_to_f32(sm.scale[k]);
+    // split: thread pair kp = tid % 128 of the slice (k = 2 kp, 2 kp + 1), tokens
+    // tid / 128 + 2 i
+    const int kp = tid & 127, k = 2 * kp, b = k >> 6, kk = k & 63;
+    const float2 sc = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sm.scale[k]));
 #pragma unroll 4
-    for (int i = 0; i < TOK; ++i) {
-      const float xv = bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(sm.x[b] + sw_off(i, kk)));
-      const float pv = __fmul_rn(xv, s);
-      const __nv_bfloat16 h = __float2bfloat16_rn(pv);
-      const __nv_bfloat16 l = __float2bfloat16_rn(pv - __bfloat162float(h));
-      *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(sm.hi) + split_off(i, k)) = h;
-      *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(sm.lo) + split_off(i, k)) = l;
+    for (int i = tid >> 7; i < TOK; i += 2) {
+      const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sm.x[b] + sw_off(i, kk)));
+      const float p0 = __fmul_rn(xv.x, sc.x), p1 = __fmul_rn(xv.y, sc.y);
+      const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+      const float2 hf = __bfloat1622float2(h);
+      const __nv_bfloat162 l = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<uint8_t*>(sm.hi) + split_off(i, k)) = h;
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<uint8_t*>(sm.lo) + split_off(i, k)) = l;
     }
     // sum of squares of x over the slice: warp w takes tokens w, w + 8, ...;
     // lane l sums k = 8l .. 8l + 7, then a butterfly over the warp
@@ -670,31 +681,30 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       for (int n = 0; n < 2; ++n)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc2[m][n][i] = 0.f;
+    // fragments by ldmatrix: lane l addresses row l % 8 of matrix l / 8
+    const int mat = lane >> 3, rr = lane & 7;
+    const uint32_t hbase = smem_u32(sm.hi), lbase = smem_u32(sm.lo);
 #pragma unroll 2
     for (int ks = 0; ks < kRcK / 16; ++ks) {
-      const int kb = ks * 16 + 2 * t4;  // this lane's low k-pair of the step
-      uint32_t bfr[2][2];
-#pragma unroll
-      for (int n = 0; n < 2; ++n) {
-        const int e = 16 * warp + 8 * n + g;
-        const uint8_t* pb = sm.proj[kb >> 6];
-        bfr[n][0] = lds_u32(pb + sw_off(e, kb & 63));
-        bfr[n][1] = lds_u32(pb + sw_off(e, (kb + 8) & 63));
+      // B: matrices (n0, k lo), (n0, k hi), (n1, k lo), (n1, k hi) of this warp's 16 experts
+      uint32_t bq[4];
+      {
+        const int e = 16 * warp + 8 * (mat >> 1) + rr, kc = (ks & 3) * 2 + (mat & 1);
+        ldsm_x4(smem_u32(sm.proj[ks >> 2]) + (uint32_t)(e * 128 + ((kc ^ rr) << 4)), bq);
       }
 #pragma unroll
       for (int m = 0; m < TOK / 16; ++m) {
-        const int r0 = 16 * m + g;
-        const uint8_t* H = reinterpret_cast<const uint8_t*>(sm.hi);
-        const uint8_t* L = reinterpret_cast<const uint8_t*>(sm.lo);
-        const uint32_t ah[4] = {lds_u32(H + split_off(r0, kb)), lds_u32(H + split_off(r0 + 8, kb)),
-                                lds_u32(H + split_off(r0, kb + 8)), lds_u32(H + split_off(r0 + 8, kb + 8))};
-        const uint32_t al[4] = {lds_u32(L + split_off(r0, kb)), lds_u32(L + split_off(r0 + 8, kb)),
-                                lds_u32(L + split_off(r0, kb + 8)), lds_u32(L + split_off(r0 + 8, kb + 8))};
+        // A: matrices (rows lo, k lo), (rows hi, k lo), (rows lo, k hi), (rows hi, k hi)
+        const int row = 16 * m + rr + 8 * (mat & 1), kc = ks * 2 + (mat >> 1);
+        const uint32_t off = (uint32_t)(row * (kRcK * 2) + ((kc ^ rr) << 4));
+        uint32_t ah[4], al[4];
+        ldsm_x4(hbase + off, ah);
+        ldsm_x4(lbase + off, al);
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
           float (&d)[4] = (ks & 1) ? acc2[m][n] : acc[m][n];
-          mma_bf16_16816(d, ah, bfr[n][0], bfr[n][1]);
-          mma_bf16_16816(d, al, bfr[n][0], bfr[n][1]);
+          mma_bf16_16816(d, ah, bq[2 * n], bq[2 * n + 1]);
+          mma_bf16_16816(d, al, bq[2 * n], bq[2 * n + 1]);
         }
       }
     }
@@ -751,6 +761,170 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   block_permute_small(a);
 }
 
+// ------------------------------------------------------------------------
+// Wide router (many tokens): a CTA owns 32 tokens and all 128 experts over
+// the whole K, streamed in blocks of 64 through an 8-deep ring (proj block
+// 128 x 64 and x block 32 x 64, both 128B-swizzled TMA boxes, and the
+// scale block by a bulk copy).  16 warps: per block every thread splits two
+// pairs of products x * scale into hi/lo bf16 (double-buffered tiles), one
+// barrier, then warp w runs the hi and lo MMAs for experts [16 (w % 8), +16)
+// and token tile w / 8.  Softmax / top-8 at the end from the logits in
+// shared memory.
+constexpr int kRwTok = 32;
+constexpr int kRwNS = 8;
+constexpr int kRwThreads = 512;
+
+struct RwSmem {
+  uint8_t proj[kRwNS][kE * 128];
+  uint8_t x[kRwNS][kRwTok * 128];
+  uint16_t scale[kRwNS][64];
+  uint16_t hi[2][kRwTok * 64];   // 128-byte rows, 16-byte chunks XOR (token & 7)
+  uint16_t lo[2][kRwTok * 64];
+  float logits[kRwTok][kE];
+  float ss[kRwTok];
+  uint64_t full[kRwNS];
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kRwThreads, 1)
+    route_wide_kernel(const __grid_constant__ CUtensorMap tm_proj, const __grid_constant__ CUtensorMap tm_x,
+                      RouteArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  RwSmem& sm = *reinterpret_cast<RwSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+  const int tok0 = blockIdx.x * kRwTok;
+  const int nkb = a.H / 64;
+  constexpr uint32_t kStageTx = kE * 128 + kRwTok * 128 + 128;
+
+  if (tid == 0) {
+    for (int i = 0; i < kRwNS; ++i) mbar_init(&sm.full[i], 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int kb) {
+    const int sl = kb % kRwNS;
+    mbar_arrive_expect_tx(&sm.full[sl], kStageTx);
+    tma_load_2d_rc(smem_u32(sm.proj[sl]), &tm_proj, kb * 64, 0, &sm.full[sl]);
+    tma_load_2d_rc(smem_u32(sm.x[sl]), &tm_x, kb * 64, tok0, &sm.full[sl]);  // rows past T read as zero
+    bulk_g2s(sm.scale[sl], a.scale + kb * 64, 128, &sm.full[sl]);
+  };
+  if (tid == 0)
+    for (int kb = 0; kb < kRwNS - 1 && kb < nkb; ++kb) issue(kb);
+
+  const int eg = warp & 7, mt = warp >> 3;  // expert group (16 experts), token tile
+  float acc[2][4];
+#pragma unroll
+  for (int n = 0; n < 2; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+  // this thread's split elements: k pair kp = lane (k = 2 kp, 2 kp + 1), tokens warp, warp + 16
+  const int kp = lane;
+  float ssq[2] = {0.f, 0.f};
+  int issued = min(kRwNS - 1, nkb);
+
+  for (int kb = 0; kb < nkb; ++kb) {
+    const int sl = kb % kRwNS, hb = kb & 1;
+    if (!mbar_wait_bounded(&sm.full[sl], (kb / kRwNS) & 1)) {
+      record_status(a.status, kStatusTimeout);
+      atomicExch(&sm.abort_flag, 1);
+    }
+    const float2 sc = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sm.scale[sl][2 * kp]));
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int r = warp + 16 * i;
+      const uint32_t off = sw_off(r, 2 * kp);
+      const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(sm.x[sl] + off));
+      ssq[i] = __fmaf_rn(xv.x, xv.x, ssq[i]);
+      ssq[i] = __fmaf_rn(xv.y, xv.y, ssq[i]);
+      const float p0 = __fmul_rn(xv.x, sc.x), p1 = __fmul_rn(xv.y, sc.y);
+      const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+      const float2 hf = __bfloat1622float2(h);
+      const __nv_bfloat162 l = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<uint8_t*>(sm.hi[hb]) + off) = h;
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<uint8_t*>(sm.lo[hb]) + off) = l;
+    }
+    __syncthreads();  // split tiles ready; the MMAs of block kb - 1 are done everywhere
+    if (sm.abort_flag) break;  // uniform: read after the barrier
+    if (tid == 0 && issued < nkb) issue(issued++);  // refills the slot of block kb - 1
+    // fragments by ldmatrix: lane l addresses row l % 8 of matrix l / 8
+    const int mat = lane >> 3, rr = lane & 7;
+    const uint32_t pb = smem_u32(sm.proj[sl]), hbase = smem_u32(sm.hi[hb]), lbase = smem_u32(sm.lo[hb]);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t bq[4];
+      {
+        const int e = 16 * eg + 8 * (mat >> 1) + rr, kc = ks * 2 + (mat & 1);
+        ldsm_x4(pb + (uint32_t)(e * 128 + ((kc ^ rr) << 4)), bq);
+      }
+      const int row = 16 * mt + rr + 8 * (mat & 1), kc = ks * 2 + (mat >> 1);
+      const uint32_t off = (uint32_t)(row * 128 + ((kc ^ rr) << 4));
+      uint32_t ah[4], al[4];
+      ldsm_x4(hbase + off, ah);
+      ldsm_x4(lbase + off, al);
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        mma_bf16_16816(acc[n], ah, bq[2 * n], bq[2 * n + 1]);
+        mma_bf16_16816(acc[n], al, bq[2 * n], bq[2 * n + 1]);
+      }
+    }
+  }
+  // sums of squares: warp w holds tokens w and w + 16 over all k (lane = k pair)
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float q2 = ssq[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q2 += __shfl_xor_sync(0xffffffffu, q2, o);
+    if (lane == 0) sm.ss[warp + 16 * i] = q2;
+  }
+#pragma unroll
+  for (int n = 0; n < 2; ++n) {
+    const int e = 16 * eg + 8 * n + 2 * t4;
+    sm.logits[16 * mt + g][e] = acc[n][0];
+    sm.logits[16 * mt + g][e + 1] = acc[n][1];
+    sm.logits[16 * mt + g + 8][e] = acc[n][2];
+    sm.logits[16 * mt + g + 8][e + 1] = acc[n][3];
+  }
+  __syncthreads();
+  if (!sm.abort_flag) {
+    // softmax / top-8: warp w finishes tokens 2w, 2w + 1
+    for (int j = 2 * warp; j < 2 * warp + 2; ++j) {
+      const int t = tok0 + j;
+      if (t >= a.T) break;
+      const float f = (1.0f / sqrtf(sm.ss[j] / (float)a.H + a.eps)) * a.inv_sqrt_h;
+      float lg[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lg[i] = sm.logits[j][lane + 32 * i] * f + (a.bias ? a.bias[lane + 32 * i] : 0.f);
+      finish_token(a, t, lg);
+    }
+  } else if (tid == 0) {
+    // let copies of a failed wait land before the CTA exits
+    for (int kb = max(0, issued - kRwNS); kb < issued; ++kb)
+      mbar_wait_bounded(&sm.full[kb % kRwNS], (kb / kRwNS) & 1, kAbortDrainNs);
+  }
+}
+
+cudaError_t launch_route_wide(const RouteArgs& a, cudaStream_t st) {
+  static int configured_dev = -1;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const int smem = (int)sizeof(RwSmem) + 1024;
+  if (configured_dev != dev) {
+    err = cudaFuncSetAttribute(route_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    configured_dev = dev;
+  }
+  CUtensorMap tm_proj, tm_x;
+  if (!encode_tma_2d(&tm_proj, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.proj, (uint64_t)a.H, kE, (uint64_t)a.H * 2, 64, kE,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tma_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, (uint64_t)a.H, (uint64_t)a.T, (uint64_t)a.H * 2, 64,
+                     kRwTok, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  route_wide_kernel<<<(a.T + kRwTok - 1) / kRwTok, kRwThreads, smem, st>>>(tm_proj, tm_x, a);
+  return cudaGetLastError();
+}
+
 template <int TOK>
 cudaError_t launch_route_cluster(const RouteArgs& a, cudaStream_t st) {
   static int configured_dev = -1;
@@ -795,6 +969,8 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   // few tokens and hidden sizes of 8 to 16 slices of 256: one cluster per 16 tokens
   if (a.few_tokens && a.H % kRcK == 0 && a.H / kRcK >= kRcMinRanks && a.H / kRcK <= kRcMaxRanks)
     return launch_route_cluster<16>(a, st);
+  // many tokens: 32 tokens per CTA over the whole K
+  if (!a.few_tokens && a.H % 64 == 0) return launch_route_wide(a, st);
   if (a.few_tokens) {
     static int configured_dev = -1;
     int dev = 0;

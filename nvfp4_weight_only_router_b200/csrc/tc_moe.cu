@@ -498,37 +498,45 @@ cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
 
 // xs[pos] = f16(x[token of sorted slot pos]) (saturating): the activations in
 // expert order and in the f16 of the MMA operands, so that every tile of the
-// expert GEMMs reads contiguous rows.  One thread per 8 elements.
+// expert GEMMs reads contiguous rows.  One warp per row: 352 16-byte chunks,
+// 11 per lane, all loads in flight before the stores.
 __global__ void __launch_bounds__(256) gather_sorted_kernel(const uint16_t* __restrict__ x,
                                                             const int* __restrict__ sorted_slot,
                                                             const int* __restrict__ meta, int T,
                                                             __half* __restrict__ xs, int* status) {
-  constexpr int per_row = kH / 8;  // 16-byte chunks per row
+  constexpr int per_row = kH / 8;              // 352
+  constexpr int per_lane = per_row / 32;       // 11
   const int S = meta[kMetaOffsets + kE];
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)S * per_row;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int pos = (int)(i / per_row), c = (int)(i % per_row);
+  const int lane = threadIdx.x & 31;
+  for (int pos = blockIdx.x * 8 + (threadIdx.x >> 5); pos < S; pos += gridDim.x * 8) {
     int tok = sorted_slot[pos] / kTopK;
     if (tok < 0 || tok >= T) {
       record_status(status, kStatusDevice);
       tok = 0;
     }
-    const uint4 v = ldg_nc_v4(x + (size_t)tok * kH + 8 * c);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * kH);
+    uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)pos * kH);
+    uint4 v[per_lane];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      o[k] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(w[k] & 0xFFFFu)), f32_to_f16_sat(bf16_bits_to_f32(w[k] >> 16)));
-    reinterpret_cast<uint4*>(xs + (size_t)pos * kH)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int i = 0; i < per_lane; ++i) v[i] = ldg_nc_v4(src + lane + 32 * i);
+#pragma unroll
+    for (int i = 0; i < per_lane; ++i) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        o[k] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(w[k] & 0xFFFFu)), f32_to_f16_sat(bf16_bits_to_f32(w[k] >> 16)));
+      __stcs(dst + lane + 32 * i, make_uint4(o[0], o[1], o[2], o[3]));
+    }
   }
 }
 
 }  // namespace
 
 cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st) {
-  const int64_t n = (int64_t)a.T * kTopK * (kH / 8);
-  int blocks = (int)((n + 255) / 256);
-  if (blocks > 4096) blocks = 4096;
+  const int64_t rows = (int64_t)a.T * kTopK;
+  int blocks = (int)((rows + 7) / 8);
+  if (blocks > 148 * 32) blocks = 148 * 32;
   gather_sorted_kernel<<<blocks, 256, 0, st>>>(a.x, a.sorted_slot, a.meta, a.T, a.xs, a.status);
   return cudaGetLastError();
 }

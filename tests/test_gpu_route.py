@@ -50,3 +50,14 @@ def test_route_ties_pick_lower_id(dev):
     x = gen.make_x(9, 4)
     ids, _ = lib.route(bf16_to_dev(x, dev), drt)
     assert (ids.cpu().numpy() == np.arange(8)[None, :]).all()
+
+
+@pytest.mark.parametrize("h,T", [(2048, 3), (2048, 40), (4096, 17), (640, 300), (384, 20), (256, 600)])
+def test_route_hidden_sizes_all_paths(dev, h, T):
+    # clusters of 8 and 16 CTAs (h = 2048, 4096), the wide kernel with an odd
+    # number of 64-wide K blocks (h = 640, T > 256), and the fallbacks for hidden
+    # sizes that are not multiples of 256 (few tokens) or too small for a cluster
+    rt = gen.make_router(20 + h, h=h)
+    drt = lib.Router.from_host(rt, dev)
+    x = gen.make_x(21 + T, T, h)
+    _check(x, rt, drt, dev)
