@@ -56,14 +56,17 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
-// Index of the E2M1 magnitude nearest to a >= 0 among {0, .5, 1, 1.5, 2, 3, 4, 6};
-// exact midpoints go to the even index; values above 6 give 7.  Each term
-// counts one grid midpoint that `a` lies above (strictly, where the midpoint
-// rounds down to an even code; inclusively where it rounds up to one).
-__device__ __forceinline__ uint32_t e2m1_magnitude_rne(float a) {
-  return (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
-         (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
-         (uint32_t)(a > 5.0f);
+// Two fp32 values -> two E2M1 codes (4-bit: sign, 2 exponent bits, 1 mantissa
+// bit) in one byte, `hi` in the high nibble: the hardware conversion rounds to
+// nearest with ties to the even code and saturates at 6, which is the grid
+// rounding of the method; the sign bit follows the value (-0 and negatives
+// that round to 0 give 0x8).
+__device__ __forceinline__ uint32_t e2m1x2_rne(float hi, float lo) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 b;\n\tcvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\tcvt.u16.u8 %0, b;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return r & 0xFFu;
 }
 
 __global__ void __launch_bounds__(256) encode_kernel(const uint16_t* __restrict__ w,
@@ -96,12 +99,17 @@ __global__ void __launch_bounds__(256) encode_kernel(const uint16_t* __restrict_
   const float d = __fmul_rn(e4m3_to_f32(sc), G);
 
   uint32_t packed[2] = {0u, 0u};
+  if (d > 0.0f) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t sign = (__float_as_uint(x[i]) >> 31) << 3;
-    uint32_t mag = 0;
-    if (d > 0.0f) mag = e2m1_magnitude_rne(fabsf(__fdiv_rn(x[i], d)));
-    packed[i >> 3] |= (sign | mag) << ((i & 7) * 4);
+    for (int i = 0; i < 16; i += 2) {
+      // element 2j in the low nibble of byte j
+      const uint32_t byte = e2m1x2_rne(__fdiv_rn(x[i + 1], d), __fdiv_rn(x[i], d));
+      packed[i >> 3] |= byte << ((i & 7) * 4);
+    }
+  } else {
+    // zero block (d = 0): only the sign bits
+#pragma unroll
+    for (int i = 0; i < 16; ++i) packed[i >> 3] |= ((__float_as_uint(x[i]) >> 31) << 3) << ((i & 7) * 4);
   }
   *reinterpret_cast<uint2*>(q + blk * 8) = make_uint2(packed[0], packed[1]);
   s[blk] = (uint8_t)sc;
