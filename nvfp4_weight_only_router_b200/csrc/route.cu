@@ -43,7 +43,9 @@ __device__ __forceinline__ void split_hi_lo(float p0, float p1, uint32_t& hi, ui
 
 // Top-8 of 128 logits held 4 per lane (expert lane + 32 i).  Ordered by
 // descending logit (= descending probability); equal logits -> lower id first.
-__device__ void finish_token(const RouteArgs& a, int t, const float (&lg)[4]) {
+// pesv[i] = per_expert_scale of expert lane + 32 i (loaded by the caller ahead
+// of time, so no global read sits on this token's critical path).
+__device__ void finish_token(const RouteArgs& a, int t, const float (&lg)[4], const float (&pesv)[4]) {
   const int lane = threadIdx.x & 31;
   float m = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
 #pragma unroll
@@ -62,7 +64,7 @@ __device__ void finish_token(const RouteArgs& a, int t, const float (&lg)[4]) {
 
   bool taken[4] = {false, false, false, false};
   int sel_id = 0;
-  float sel_p = 0.f, psum = 0.f;
+  float sel_p = 0.f, sel_pes = 0.f, psum = 0.f;
   for (int r = 0; r < kTopK; ++r) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
@@ -83,24 +85,36 @@ __device__ void finish_token(const RouteArgs& a, int t, const float (&lg)[4]) {
       }
     }
     const int owner = bi & 31, slot = bi >> 5;
-    float pw = 0.f;
+    float pw = 0.f, pe = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       if (lane == owner && slot == i) {
         taken[i] = true;
         pw = p[i];
+        pe = pesv[i];
       }
     pw = __shfl_sync(0xffffffffu, pw, owner);
+    pe = __shfl_sync(0xffffffffu, pe, owner);
     psum += pw;
     if (lane == r) {
       sel_id = bi;
       sel_p = pw;
+      sel_pes = pe;
     }
   }
   if (lane < kTopK) {
-    const float pes = bf16_bits_to_f32(a.pes[sel_id]);
     a.ids[(size_t)t * kTopK + lane] = sel_id;
-    a.wts[(size_t)t * kTopK + lane] = (sel_p / psum) * pes;
+    a.wts[(size_t)t * kTopK + lane] = (sel_p / psum) * sel_pes;
+  }
+}
+
+// per_expert_scale and logit bias of experts lane + 32 i
+__device__ __forceinline__ void load_expert_consts(const RouteArgs& a, float (&pesv)[4], float (&bv)[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    pesv[i] = bf16_bits_to_f32(__ldg(a.pes + lane + 32 * i));
+    bv[i] = a.bias ? __ldg(a.bias + lane + 32 * i) : 0.f;
   }
 }
 
@@ -328,13 +342,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   }
 
   // softmax / top-8: warp w handles tokens 2w, 2w+1 of the tile
+  float pesv[4], bv_unused[4];
+  load_expert_consts(a, pesv, bv_unused);
   for (int j = 0; j < 2; ++j) {
     const int t = tile * 16 + warp * 2 + j;
     if (t >= a.T) break;
     float lg[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) lg[i] = __ldcg(a.logits + (size_t)t * kE + lane + 32 * i);
-    finish_token(a, t, lg);
+    finish_token(a, t, lg, pesv);
   }
 
   if (a.meta == nullptr) return;
@@ -489,13 +505,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_staged_kernel(RouteArgs a
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  float pesv[4], bv_unused[4];
+  load_expert_consts(a, pesv, bv_unused);
   for (int j = 0; j < 2; ++j) {
     const int t = tok0 + warp * 2 + j;
     if (t >= a.T) break;
     float lg[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) lg[i] = __ldcg(a.logits + (size_t)t * kE + lane + 32 * i);
-    finish_token(a, t, lg);
+    finish_token(a, t, lg, pesv);
   }
   if (a.meta == nullptr) return;
   // few tokens: the last token tile to finish also runs the permutation
@@ -558,11 +576,6 @@ __device__ __forceinline__ uint32_t map_shared(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
 __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a0, float a1) {
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a0), "f"(a1) : "memory");
 }
@@ -577,11 +590,6 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
       : "r"(addr)
       : "memory");
-}
-__device__ __forceinline__ uint32_t lds_u32(const void* p) {
-  uint32_t v;
-  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
 }
 __device__ __forceinline__ void tma_load_2d_rc(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
   asm volatile(
@@ -610,6 +618,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   const int r = (int)cluster_ctarank(), nr = a.H / kRcK;
   const int tok0 = blockIdx.y * TOK;
   const int k0 = r * kRcK;
+  float pesv[4], biasv[4];  // read now; used by the warps that finish tokens
+  load_expert_consts(a, pesv, biasv);
 
   if (tid == 0) {
     mbar_init(&sm.bar, 1);
@@ -739,8 +749,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     }
     const float f = (1.0f / sqrtf(ssum / (float)a.H + a.eps)) * a.inv_sqrt_h;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) lg[i] = lg[i] * f + (a.bias ? a.bias[lane + 32 * i] : 0.f);
-    finish_token(a, t, lg);
+    for (int i = 0; i < 4; ++i) lg[i] = lg[i] * f + biasv[i];
+    finish_token(a, t, lg, pesv);
   }
   __syncthreads();
   cluster_sync_all();  // no CTA exits while peers may still store into it
@@ -794,6 +804,8 @@ __global__ void __launch_bounds__(kRwThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
   const int tok0 = blockIdx.x * kRwTok;
   const int nkb = a.H / 64;
+  float pesv[4], biasv[4];  // read now; used by the warps that finish tokens
+  load_expert_consts(a, pesv, biasv);
   constexpr uint32_t kStageTx = kE * 128 + kRwTok * 128 + 128;
 
   if (tid == 0) {
@@ -894,8 +906,8 @@ __global__ void __launch_bounds__(kRwThreads, 1)
       const float f = (1.0f / sqrtf(sm.ss[j] / (float)a.H + a.eps)) * a.inv_sqrt_h;
       float lg[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) lg[i] = sm.logits[j][lane + 32 * i] * f + (a.bias ? a.bias[lane + 32 * i] : 0.f);
-      finish_token(a, t, lg);
+      for (int i = 0; i < 4; ++i) lg[i] = sm.logits[j][lane + 32 * i] * f + biasv[i];
+      finish_token(a, t, lg, pesv);
     }
   } else if (tid == 0) {
     // let copies of a failed wait land before the CTA exits

@@ -73,6 +73,7 @@ struct alignas(1024) SSmem {
   uint8_t x[kNS][kXBytes];
   uint64_t full[kNS], empty[kNS];
   int unit_prefix[kE + 1];
+  int offs[kE + 1];                // per-expert slot offsets (copied from meta once)
   int abort_flag;
   int issued;       // stages issued
 };
@@ -82,9 +83,10 @@ struct Unit {
 };
 
 // Unit u of the launch: expert by binary search over the per-expert unit
-// prefix, then (token group, row block) with the row block fastest.
+// prefix, then (token group, row block) with the row block fastest.  All
+// reads are shared memory (offs = the per-expert slot offsets).
 template <int KIND>
-__device__ __forceinline__ Unit decode_unit(const int* prefix, const int* meta, int u) {
+__device__ __forceinline__ Unit decode_unit(const int* prefix, const int* offs, int u) {
   int lo = 0, hi = kE - 1;  // largest e with prefix[e] <= u
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -95,8 +97,8 @@ __device__ __forceinline__ Unit decode_unit(const int* prefix, const int* meta, 
   const int local = u - prefix[lo];
   r.tg = local / SCfg<KIND>::NJ;
   r.j = local % SCfg<KIND>::NJ;
-  r.off = meta[kMetaOffsets + lo];
-  const int cnt = meta[kMetaOffsets + lo + 1] - r.off;
+  r.off = offs[lo];
+  const int cnt = offs[lo + 1] - r.off;
   r.nvalid = min(kUTok, cnt - r.tg * kUTok);
   return r;
 }
@@ -159,7 +161,7 @@ __device__ __forceinline__ void mma_chunk(float (&acc)[NNT][CH][4], const uint4&
 // prefetch the e4m3 scales three stages ahead, once to compute.
 template <int KIND>
 struct ScalePrefetch {
-  const int* meta;
+  const int* offs;           // per-expert slot offsets (shared memory)
   const uint8_t* scales;     // gate_up or down scale matrix
   const int* prefix;
   int begin, n_local, rowA, rowB, q;
@@ -168,7 +170,7 @@ struct ScalePrefetch {
 
   __device__ __forceinline__ void set_unit() {
     if (u >= n_local) return;
-    const Unit U = decode_unit<KIND>(prefix, meta, begin + u);
+    const Unit U = decode_unit<KIND>(prefix, offs, begin + u);
     if (KIND == kGateUp) {
       const size_t g0 = (size_t)U.e * (2 * kI) + (size_t)U.j * 64;  // first gate row of the unit
       sa = scales + (g0 + rowA) * kGuScaleRow;                      // rowA < 64: gate row
@@ -219,6 +221,19 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
                                              Lane& L, ScalePrefetch<KIND>& pf, int wq, int g, int q) {
   using C = SCfg<KIND>;
   constexpr int CH = 4 / NNT;  // independent accumulator chains per n-tile
+  // the epilogue's global reads, issued now so their latency hides behind the
+  // unit's stages: the expert's global scale and (down) the routing weight of
+  // each of this lane's token columns
+  const float G = KIND == kGateUp ? __ldg(p.gu_g + U.e) : __ldg(p.dn_g + U.e);
+  float wgt[NNT][2];
+#pragma unroll
+  for (int nt = 0; nt < NNT; ++nt)
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+      const int n = nt * 8 + 2 * q + c2;
+      wgt[nt][c2] = 0.f;
+      if (KIND == kDown && n < U.nvalid) wgt[nt][c2] = __ldg(p.wts + __ldg(p.sorted_slot + U.off + U.tg * kUTok + n));
+    }
   float acc[NNT][CH][4];
 #pragma unroll
   for (int nt = 0; nt < NNT; ++nt)
@@ -251,7 +266,6 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
   }
 
   // ------------------------------------------------------------ epilogue
-  const float G = KIND == kGateUp ? p.gu_g[U.e] : p.dn_g[U.e];
 #pragma unroll
   for (int nt = 0; nt < NNT; ++nt) {
     float v[4];
@@ -271,10 +285,10 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
         const int unit = U.j * 64 + 8 * wq + g;
         p.h[(size_t)pos * kI + unit] = f32_to_f16_sat(gelu_tanh(G * v[c2]) * (G * v[2 + c2]));
       } else {
-        const float wgt = p.wts[p.sorted_slot[pos]] * G;
+        const float wg = wgt[nt][c2] * G;
         const int row0 = U.j * kURows + 16 * wq + g;
-        p.obuf[(size_t)pos * kH + row0] = v[c2] * wgt;
-        p.obuf[(size_t)pos * kH + row0 + 8] = v[2 + c2] * wgt;
+        p.obuf[(size_t)pos * kH + row0] = v[c2] * wg;
+        p.obuf[(size_t)pos * kH + row0 + 8] = v[2 + c2] * wg;
       }
     }
   }
@@ -315,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 31) sm.unit_prefix[kE] = incl;
   }
+  for (int i = threadIdx.x; i <= kE; i += kThreads) sm.offs[i] = p.meta[kMetaOffsets + i];
   if (warp == kProdWarp && lane == 0) {
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&sm.full[s], 1);
@@ -340,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nm = (2 * pp + 1 < n_local) ? 2 : 1;
         Unit U[2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) U[m] = decode_unit<KIND>(sm.unit_prefix, p.meta, begin + 2 * pp + (m < nm ? m : 0));
+        for (int m = 0; m < 2; ++m) U[m] = decode_unit<KIND>(sm.unit_prefix, sm.offs, begin + 2 * pp + (m < nm ? m : 0));
         for (int kc = 0; kc < C::KC && ok; ++kc) {
 #pragma unroll
           for (int m = 0; m < 2; ++m) {
@@ -387,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       L.xo[s2] = (uint32_t)(g * kXRowBytes + 128 * q + (((4 * s2) ^ k) << 4));
     }
     ScalePrefetch<KIND> pf;
-    pf.meta = p.meta;
+    pf.offs = sm.offs;
     pf.scales = KIND == kGateUp ? p.gu_s : p.dn_s;
     pf.prefix = sm.unit_prefix;
     pf.begin = begin;
@@ -402,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     L.sq[1] = pf.next();
     L.sq[2] = pf.next();
     for (int u = grp; u < n_local; u += kGroups) {
-      const Unit U = decode_unit<KIND>(sm.unit_prefix, p.meta, begin + u);
+      const Unit U = decode_unit<KIND>(sm.unit_prefix, sm.offs, begin + u);
       const bool ok = U.nvalid > 8 ? consume_unit<KIND, 2>(sm, p, U, u, n_local, L, pf, wq, g, q)
                                    : consume_unit<KIND, 1>(sm, p, U, u, n_local, L, pf, wq, g, q);
       if (!ok) break;
