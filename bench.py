@@ -37,6 +37,11 @@ EXPERT_BYTES = GU_EXPERT_BYTES + DN_EXPERT_BYTES        # 3,345,416
 ROUTER_BYTES = 128 * 2816 * 2 + 2816 * 2 + 128 * 2       # 726,784 (bf16 proj, scale, pes)
 FLUSH_BYTES = 256 << 20
 
+# DRAM read + write per launch of the dominant kernel, from the ncu captures
+# summarised in profiles/ (stream_gemv_decode64.md, tc_moe_prefill4096.md);
+# None where no capture of the current kernel exists
+TRAFFIC_BYTES = {"decode64": 287.66e6, "prefill4096": 515.49e6}
+
 WORKLOADS = {
     "decode64": {"T": 64, "layers": 1, "zipf": False,
                  "desc": "one MoE layer (H=2816, E=128, top-8, I=704, NVFP4 experts), decode T=64"},
@@ -399,12 +404,14 @@ def run_ours(args, wl, rank, world, local_rank):
         if T >= 1024:
             ach = gu_flops / (gu_ms.mean() / 1e3) / 1e12
             roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM + GELU", "achieved": ach,
-                    "peak": tc_peak_sus, "unit": "TFLOP/s", "traffic": None, "peak_kind": peak_kind + " sustained",
+                    "peak": tc_peak_sus, "unit": "TFLOP/s", "traffic": TRAFFIC_BYTES.get(args.workload),
+                    "peak_kind": peak_kind + " sustained",
                     "algorithmic_per_launch": gu_flops}
         else:
             ach = gu_bytes.sum() / (gu_ms.sum() / 1e3) / 1e9
             roof = {"bound": "hbm", "kernel": "gate_up grouped GEMV + GELU", "achieved": ach,
-                    "peak": hbm_peak, "unit": "GB/s", "traffic": None, "peak_kind": peak_kind,
+                    "peak": hbm_peak, "unit": "GB/s", "traffic": TRAFFIC_BYTES.get(args.workload),
+                    "peak_kind": peak_kind,
                     "algorithmic_per_launch": float(gu_bytes.mean())}
         roof["frac"] = roof["achieved"] / roof["peak"]
         step_bytes = n_act * EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2
