@@ -301,8 +301,11 @@ def run_ours(args, wl, rank, world, local_rank):
         def prepare(i):
             xs.copy_(x_pool[i % n_pool])
 
-        # route, permute, gate_up, down, combine per layer (+ the chain's rmsnorm kernels)
-        kernels_per_step = 5 * len(layers) + (len(layers) + 1 if len(layers) > 1 else 0)
+        # per layer: route (with the permutation when T*8 <= 1024, else two
+        # permutation kernels), gather, gate_up, down, combine; plus the
+        # chain's rmsnorm kernels
+        per_layer = 5 if T * 8 <= 1024 else 7
+        kernels_per_step = per_layer * len(layers) + (len(layers) + 1 if len(layers) > 1 else 0)
 
     # -------- warm-up (at least W steps and at least 1 s, so the clock sampler sees load)
     sampler = ClockSampler(physical_gpu_index(local_rank))
