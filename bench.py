@@ -221,15 +221,16 @@ def run_ours(args, wl, rank, world, local_rank):
         q = torch.empty((128, 1408, 1408), dtype=torch.uint8, device=dev)
         s = torch.empty((128, 1408, 176), dtype=torch.uint8, device=dev)
         g = torch.empty((128,), dtype=torch.float32, device=dev)
-        ws = torch.empty(512, dtype=torch.uint8, device=dev)
         from nvfp4_weight_only_router_b200 import capi
+        ws_bytes = capi.nvfp4_quantize_workspace_bytes(128, 1408, 2816)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
         def step(i):
             capi.check(capi.nvfp4_quantize(wd.data_ptr(), 128, 1408, 2816, q.data_ptr(), s.data_ptr(),
-                                           g.data_ptr(), ws.data_ptr(), 512,
+                                           g.data_ptr(), ws.data_ptr(), ws_bytes,
                                            torch.cuda.current_stream().cuda_stream))
         algo_bytes = wd.numel() * 2 + q.numel() + s.numel() + 128 * 4
-        kernels_per_step = 2
+        kernels_per_step = 1  # the single-pass kernel (the clearing of its counters is a memset)
     else:
         layers = []
         seeds = [0] if wl["layers"] == 1 else gen.layer_seed_plan(wl["layers"])
@@ -388,7 +389,7 @@ def run_ours(args, wl, rank, world, local_rank):
     if args.workload == "quantize":
         value = world * algo_bytes * args.steps / (total_ms / 1e3) / 1e9
         unit = "GB/s"
-        roof = {"bound": "hbm", "kernel": "nvfp4_quantize (amax + encode)",
+        roof = {"bound": "hbm", "kernel": "quantize_fused_kernel (single pass: amax + encode)",
                 "achieved": algo_bytes / (ms_per_step / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                 "traffic": None, "peak_kind": peak_kind}
         roof["frac"] = roof["achieved"] / roof["peak"]

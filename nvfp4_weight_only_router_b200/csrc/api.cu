@@ -19,7 +19,9 @@ constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {};
 std::mutex g_status_mu;
 
-int* device_status_ptr() {
+}  // namespace
+
+int* nvfp4moe::device_status_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_status_mu);
@@ -30,6 +32,8 @@ int* device_status_ptr() {
   }
   return g_status_ptr[dev];
 }
+
+namespace {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -204,7 +208,8 @@ static nvfp4_status check_quant_dims(int64_t E, int64_t N, int64_t K) {
 
 size_t nvfp4_quantize_workspace_bytes(int64_t E, int64_t N, int64_t K) {
   if (check_quant_dims(E, N, K) != NVFP4_OK) return 0;
-  return round_up(sizeof(uint32_t) * (size_t)E, 256);
+  // E amax words + 3 arrival counters of the single-pass kernel
+  return round_up(sizeof(uint32_t) * (size_t)(E + 3), 256);
 }
 
 nvfp4_status nvfp4_quantize(const void* w, int64_t E, int64_t N, int64_t K, uint8_t* q, uint8_t* s,
@@ -217,7 +222,8 @@ nvfp4_status nvfp4_quantize(const void* w, int64_t E, int64_t N, int64_t K, uint
   if (!ws || ws_bytes < nvfp4_quantize_workspace_bytes(E, N, K)) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
   return cuda_status(launch_quantize(static_cast<const uint16_t*>(w), E, N, K, q, s, g,
-                                     static_cast<uint32_t*>(ws), as_stream(stream)));
+                                     static_cast<uint32_t*>(ws), (int64_t)(ws_bytes / sizeof(uint32_t)),
+                                     device_status_ptr(), as_stream(stream)));
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* s, const float* g, int64_t E,

@@ -8,8 +8,13 @@
 
 namespace nvfp4moe {
 
+// amax_ws: ws_words zero-initialised-by-the-call words; E + 3 or more enables
+// the single-pass kernel (E amax words + 3 arrival counters), else two passes
 cudaError_t launch_quantize(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* q,
-                            uint8_t* s, float* g, uint32_t* amax_ws, cudaStream_t st);
+                            uint8_t* s, float* g, uint32_t* amax_ws, int64_t ws_words, int* status,
+                            cudaStream_t st);
+// the library's device status word of the current device (null on failure)
+int* device_status_ptr();
 cudaError_t launch_dequantize(const uint8_t* q, const uint8_t* s, const float* g, int64_t E,
                               int64_t N, int64_t K, float* out, cudaStream_t st);
 

@@ -7,8 +7,24 @@
 // the E2M1 value nearest to w / d, ties to the even code, saturating at 6, with
 // the sign bit of w.  Each step is one correctly rounded fp32 operation.
 //
-// Pass 1 (amax_kernel) reduces |w| per tensor; pass 2 (encode_kernel) encodes
-// one 16-element block per thread with 32-byte loads and 8-byte stores.
+// Main path (quantize_fused_kernel): one cooperative launch, one CTA per SM,
+// reads every weight from HBM once.  Each CTA owns a contiguous 1/n of every
+// tensor and streams its pieces of tensors e .. e+3 into four shared-memory
+// buffers (bulk asynchronous copies).  Per tensor it reduces |w| over its
+// piece, publishes the maximum (atomicMax) and arrives on a counter; once all
+// CTAs have arrived it encodes its piece from shared memory.  The compute
+// warps reduce two tensors ahead of the one they encode, and a control warp
+// does the global publishing and waiting, so neither the wait nor the copies
+// of later tensors hold the compute warps up.  Every wait is bounded.
+// Fallback (tensors too large for the buffers, too small to split, or no room
+// for the counters): amax_kernel reduces |w| per tensor, then encode_kernel
+// encodes one 16-element block per thread.
+//
+// The element step avoids a division per element: with r = 1/d (correctly
+// rounded), the quotients w * r * (1 -+ 2^-20) bracket the correctly rounded
+// w / d, and E2M1 rounding is monotone, so when both bracket ends give the
+// same code that code is the one of w / d.  Blocks where they differ (a
+// quotient within ~2^-20 of a rounding threshold) take the exact division.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -69,6 +85,125 @@ __device__ __forceinline__ uint32_t e2m1x2_rne(float hi, float lo) {
   return r & 0xFFu;
 }
 
+// Eight fp32 values -> eight E2M1 codes (same rounding as e2m1x2_rne), element
+// i in nibble i of the result (element 2j in the low nibble of byte j).
+__device__ __forceinline__ uint32_t e2m1x8_rne(const float (&x)[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
+  return r;
+}
+
+// Approximate reciprocal (relative error at most 2^-23; normal inputs).
+__device__ __forceinline__ float rcp_approx(float d) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+  return r;
+}
+
+// Per-tensor constants of the block encoder: G = amax / 2688 (one correctly
+// rounded division) and k ~ 1 / (6 G) for the bracketed scale step.
+struct TensorScale {
+  float G, k_lo, k_hi;
+  bool fast;  // k finite: the bracketed scale step applies
+};
+
+__device__ __forceinline__ TensorScale tensor_scale(float amax) {
+  TensorScale t;
+  t.G = __fdiv_rn(amax, 2688.0f);
+  const float g6 = __fmul_rn(6.0f, t.G);
+  t.fast = g6 >= 1.17549435e-38f;
+  const float k = t.fast ? __fdiv_rn(1.0f, g6) : 0.0f;  // 1 / (6 G), relative error <= 2^-23
+  t.k_lo = __fmul_rn(k, 0.99999904632568359375f);      // 1 - 2^-20
+  t.k_hi = __fmul_rn(k, 1.00000095367431640625f);      // 1 + 2^-20
+  return t;
+}
+
+// Encode one block of 16 bf16 values (8 words, element 2j in the low half of
+// word j): returns the e4m3 scale code and the 16 E2M1 codes packed two per
+// byte (element 2j in the low nibble).
+//
+// The defined steps are t = (amax_b / 6) / G and x = w / d, each a correctly
+// rounded division, then monotone roundings (E4M3 RNE-satfinite of t, E2M1
+// RNE of x).  Each quotient is bracketed instead: the product with an
+// approximate reciprocal scaled by 1 -+ 2^-20 lies strictly below / above the
+// correctly rounded quotient (the approximations err by at most ~2^-22), so
+// when both ends round to the same code, so does the exact quotient.  Where
+// they differ (a quotient within ~2^-20 of a rounding threshold) the block
+// takes the correctly rounded divisions.
+__device__ __forceinline__ uint32_t encode_block16(const uint32_t (&pair)[8], const TensorScale& ts, uint2& codes) {
+  float x[16];
+  uint32_t key2 = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    x[2 * j] = bf16_bits_to_f32(pair[j] & 0xFFFFu);
+    x[2 * j + 1] = __uint_as_float(pair[j] & 0xFFFF0000u);
+    key2 = __vmaxu2(key2, pair[j] & 0x7FFF7FFFu);
+  }
+  const uint32_t key = max(key2 & 0xFFFFu, key2 >> 16);
+  const float amax_b = __uint_as_float(key << 16);
+  const float G = ts.G;
+  uint32_t sc = 0;
+  if (G > 0.0f) {
+    bool done = false;
+    if (ts.fast) {
+      uint16_t two;
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+          : "=h"(two)
+          : "f"(__fmul_rn(amax_b, ts.k_hi)), "f"(__fmul_rn(amax_b, ts.k_lo)));
+      sc = two & 0xFFu;
+      done = (uint32_t)(two >> 8) == sc;
+    }
+    if (!done) sc = f32_to_e4m3_satfinite(__fdiv_rn(__fdiv_rn(amax_b, 6.0f), G));
+  }
+  const float d = __fmul_rn(e4m3_to_f32(sc), G);
+
+  uint32_t packed[2] = {0u, 0u};
+  if (d > 0.0f) {
+    bool exact = false;
+    if (d >= 1.17549435e-38f) {  // normal d: 1/d is finite
+      const float r = rcp_approx(d);
+      const float rl = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
+      const float rh = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
+      uint32_t hi[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float a[8], b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          a[i] = __fmul_rn(x[8 * h + i], rl);
+          b[i] = __fmul_rn(x[8 * h + i], rh);
+        }
+        packed[h] = e2m1x8_rne(a);
+        hi[h] = e2m1x8_rne(b);
+      }
+      exact = packed[0] == hi[0] && packed[1] == hi[1];
+    }
+    if (!exact) {
+      // a quotient close to a rounding threshold (or a subnormal d): the
+      // correctly rounded division decides
+      packed[0] = packed[1] = 0u;
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        const uint32_t byte = e2m1x2_rne(__fdiv_rn(x[i + 1], d), __fdiv_rn(x[i], d));
+        packed[i >> 3] |= byte << ((i & 7) * 4);
+      }
+    }
+  } else {
+    // zero block (d = 0): only the sign bits
+#pragma unroll
+    for (int i = 0; i < 16; ++i) packed[i >> 3] |= ((__float_as_uint(x[i]) >> 31) << 3) << ((i & 7) * 4);
+  }
+  codes = make_uint2(packed[0], packed[1]);
+  return sc;
+}
+
 __global__ void __launch_bounds__(256) encode_kernel(const uint16_t* __restrict__ w,
                                                      int64_t blocks_per_expert, int64_t n_blocks,
                                                      const uint32_t* __restrict__ amax_bits,
@@ -77,42 +212,194 @@ __global__ void __launch_bounds__(256) encode_kernel(const uint16_t* __restrict_
   const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (blk >= n_blocks) return;
   const int64_t e = blk / blocks_per_expert;
-  const float amax = __uint_as_float(amax_bits[e]);
-  const float G = __fdiv_rn(amax, 2688.0f);
-  if (blk == e * blocks_per_expert) g[e] = G;
+  const TensorScale ts = tensor_scale(__uint_as_float(amax_bits[e]));
+  if (blk == e * blocks_per_expert) g[e] = ts.G;
 
   const uint4* src = reinterpret_cast<const uint4*>(w) + blk * 2;
   uint4 v0 = ldg_nc_v4(src), v1 = ldg_nc_v4(src + 1);
-  uint32_t pair[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-  float x[16];
-  uint32_t key = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    x[2 * j] = bf16_bits_to_f32(pair[j] & 0xFFFFu);
-    x[2 * j + 1] = bf16_bits_to_f32(pair[j] >> 16);
-    key = max(key, bf16_abs_key(pair[j] & 0xFFFFu));
-    key = max(key, bf16_abs_key(pair[j] >> 16));
-  }
-  const float amax_b = __uint_as_float(key << 16);
-  uint32_t sc = 0;
-  if (G > 0.0f) sc = f32_to_e4m3_satfinite(__fdiv_rn(__fdiv_rn(amax_b, 6.0f), G));
-  const float d = __fmul_rn(e4m3_to_f32(sc), G);
+  const uint32_t pair[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  uint2 codes;
+  const uint32_t sc = encode_block16(pair, ts, codes);
+  *reinterpret_cast<uint2*>(q + blk * 8) = codes;
+  s[blk] = (uint8_t)sc;
+}
 
-  uint32_t packed[2] = {0u, 0u};
-  if (d > 0.0f) {
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      // element 2j in the low nibble of byte j
-      const uint32_t byte = e2m1x2_rne(__fdiv_rn(x[i + 1], d), __fdiv_rn(x[i], d));
-      packed[i >> 3] |= byte << ((i & 7) * 4);
+// ------------------------------------------------------- single-pass path
+constexpr int kQThreads = 1024;                // warp 0: control; warps 1..31: compute
+constexpr int kQCompute = kQThreads - 32;
+constexpr int kQBufs = 4;                      // tensors e (encoding), e+1, e+2 (reduced), e+3 (loading)
+constexpr int kQHeader = 1024;                 // barriers, reduction slots, tensor constants, flags
+constexpr int kQMaxPiece = 54 * 1024;          // bytes per buffer (1728 blocks)
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// amax_ws: [E] amax bit patterns, then 3 arrival counters (tensor e counts on
+// counter e % 3, which receives the arrivals of e, e+3, ...); all zero on
+// entry.  Launched cooperatively (every CTA resident), one CTA per SM.
+//
+// Per CTA, tensor e lives in buffer e % 4.  The compute warps reduce |w| over
+// tensor e+2's piece while the control thread (warp 0, lane 0) publishes
+// tensor e's maximum, waits for every CTA's, and hands the tensor constants
+// back; so the global round trips overlap the compute warps' work:
+//   control: part(e+1) -> atomicMax, arrive on the counter of e+1 -> wait for
+//            all CTAs' arrivals on e -> constants of e -> scale(e) ->
+//            [free(e-1)] -> copy of e+3
+//   compute: full(e+2) -> reduce -> part(e+2) -> scale(e) -> encode e -> free(e)
+// A CTA publishes e+1 only after all CTAs published e-1, so counters modulo 3
+// never mix tensors that are both in flight.
+__global__ void __launch_bounds__(kQThreads, 1)
+    quantize_fused_kernel(const uint16_t* __restrict__ w, int E, int64_t bpe, uint32_t* amax_ws,
+                          uint8_t* __restrict__ q, uint8_t* __restrict__ s, float* __restrict__ g, int* status) {
+  extern __shared__ __align__(128) uint8_t qsm[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsm);        // copy landed
+  uint64_t* part = full + kQBufs;                           // compute warps' maxima written
+  uint64_t* scl = part + kQBufs;                            // tensor constants published
+  uint64_t* freeb = scl + kQBufs;                           // buffer fully read
+  uint32_t (*red)[32] = reinterpret_cast<uint32_t(*)[32]>(qsm + 128);          // [kQBufs][31]
+  TensorScale* ts_sh = reinterpret_cast<TensorScale*>(qsm + 128 + kQBufs * 128);  // [kQBufs]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(qsm + 960);
+  uint8_t* buf0 = qsm + kQHeader;
+  uint32_t* ctr = amax_ws + E;
+  const int n = gridDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t b0 = (int64_t)blockIdx.x * bpe / n, b1 = (int64_t)(blockIdx.x + 1) * bpe / n;
+  const int nb = (int)(b1 - b0);              // this CTA's blocks of every tensor
+  const uint32_t piece = (uint32_t)nb * 32u;  // bytes
+
+  if (tid == 0) {
+    for (int b = 0; b < kQBufs; ++b) {
+      mbar_init(&full[b], 1);
+      mbar_init(&part[b], kQCompute / 32);
+      mbar_init(&scl[b], 1);
+      mbar_init(&freeb[b], kQCompute / 32);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto fail = [&]() {
+    *abort_flag = 1;
+    record_status(status, kStatusTimeout);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ control
+    if (lane == 0) {
+      int issued = 0;
+      auto issue = [&](int t) {  // tensor t's piece into buffer t % 4
+        uint64_t* bar = &full[t % kQBufs];
+        if (piece > 0) {
+          mbar_arrive_expect_tx(bar, piece);
+          bulk_g2s(buf0 + (size_t)(t % kQBufs) * kQMaxPiece, w + ((size_t)t * bpe + b0) * 16, piece, bar);
+        } else {
+          mbar_arrive(bar);
+        }
+        issued = t + 1;
+      };
+      for (int t = 0; t < kQBufs - 1 && t < E; ++t) issue(t);
+      // publish tensor t's maximum once the compute warps have reduced it
+      auto contribute = [&](int t) -> bool {
+        const int b = t % kQBufs;
+        if (*abort_flag || !mbar_wait_bounded(&part[b], (t / kQBufs) & 1)) return false;
+        uint32_t m = 0;
+        for (int j = 0; j < kQCompute / 32; ++j) m = max(m, red[b][j]);
+        atomicMax(amax_ws + t, m << 16);  // fp32 bit pattern of the bf16 amax
+        red_release_add(ctr + t % 3, 1u);
+        return true;
+      };
+      if (!contribute(0)) fail();
+      for (int e = 0; e < E && !*abort_flag; ++e) {
+        const int b = e % kQBufs;
+        const uint32_t target = (uint32_t)n * (uint32_t)(e / 3 + 1);
+        uint32_t c = ld_acquire_u32(ctr + e % 3);  // in flight while tensor e+1 is published
+        if (e + 1 < E && !contribute(e + 1)) {
+          fail();
+          break;
+        }
+        if (c < target) {
+          const uint64_t t0 = globaltimer_ns();
+          while ((c = ld_acquire_u32(ctr + e % 3)) < target)
+            if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+        }
+        if (c < target) {
+          fail();
+          break;
+        }
+        ts_sh[b] = tensor_scale(__uint_as_float(__ldcg(amax_ws + e)));
+        if (blockIdx.x == 0) g[e] = ts_sh[b].G;
+        mbar_arrive(&scl[b]);
+        const int t = e + kQBufs - 1;
+        if (t < E) {
+          if (t >= kQBufs && !mbar_wait_bounded(&freeb[t % kQBufs], ((t - kQBufs) / kQBufs) & 1)) {
+            fail();
+            break;
+          }
+          issue(t);
+        }
+      }
+      if (*abort_flag) {
+        // let the copies still in flight land before exiting
+        for (int t = issued - kQBufs < 0 ? 0 : issued - kQBufs; t < issued; ++t)
+          mbar_wait_bounded(&full[t % kQBufs], (t / kQBufs) & 1, kAbortDrainNs);
+      }
     }
   } else {
-    // zero block (d = 0): only the sign bits
+    // ------------------------------------------------------------ compute
+    const int ct = tid - 32, cw = warp - 1;
+    auto reduce = [&](int t) -> bool {  // |w| over tensor t's piece -> red[t % 4][cw]
+      const int b = t % kQBufs;
+      if (!mbar_wait_bounded(&full[b], (t / kQBufs) & 1)) return false;
+      const uint4* v = reinterpret_cast<const uint4*>(buf0 + (size_t)b * kQMaxPiece);
+      uint32_t m = 0;
+      for (int i = ct; i < nb * 2; i += kQCompute) {
+        const uint4 u = v[i];
+        m = __vmaxu2(m, __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
+                                 __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu)));
+      }
+      m = max(m & 0xFFFFu, m >> 16);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) packed[i >> 3] |= ((__float_as_uint(x[i]) >> 31) << 3) << ((i & 7) * 4);
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) {
+        red[b][cw] = m;
+        mbar_arrive(&part[b]);
+      }
+      return true;
+    };
+    bool ok = reduce(0) && (E < 2 || reduce(1));
+    for (int e = 0; e < E && ok; ++e) {
+      if (e + 2 < E && !reduce(e + 2)) {
+        ok = false;
+        break;
+      }
+      const int b = e % kQBufs;
+      if (!mbar_wait_bounded(&scl[b], (e / kQBufs) & 1)) {
+        ok = false;
+        break;
+      }
+      const TensorScale ts = ts_sh[b];
+      const uint4* v = reinterpret_cast<const uint4*>(buf0 + (size_t)b * kQMaxPiece);
+      const size_t gb0 = (size_t)e * bpe + b0;
+      for (int lb = ct; lb < nb; lb += kQCompute) {
+        const uint4 v0 = v[2 * lb], v1 = v[2 * lb + 1];
+        const uint32_t pair[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint2 codes;
+        const uint32_t sc = encode_block16(pair, ts, codes);
+        *reinterpret_cast<uint2*>(q + (gb0 + lb) * 8) = codes;
+        s[gb0 + lb] = (uint8_t)sc;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&freeb[b]);
+    }
+    if (!ok && lane == 0) fail();
   }
-  *reinterpret_cast<uint2*>(q + blk * 8) = make_uint2(packed[0], packed[1]);
-  s[blk] = (uint8_t)sc;
+  __syncthreads();
 }
 
 // w = e2m1 * e4m3 * G rounded once to fp32: e2m1 * e4m3 is exact in f16/f32,
@@ -146,16 +433,48 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
 }
 
 cudaError_t launch_quantize(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* q,
-                            uint8_t* s, float* g, uint32_t* amax_ws, cudaStream_t st) {
-  cudaError_t err = cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * E, st);
-  if (err != cudaSuccess) return err;
+                            uint8_t* s, float* g, uint32_t* amax_ws, int64_t ws_words, int* status,
+                            cudaStream_t st) {
   const int64_t per = N * K;
+  const int64_t bpe = per / 16;
+  int dev = 0, sms = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (err != cudaSuccess) return err;
+  // single pass: the largest piece must fit a buffer, every CTA should get a
+  // few blocks, and the workspace must hold the arrival counters
+  const bool fused = ws_words >= E + 3 && E <= (int64_t(1) << 24) && bpe >= 8 * (int64_t)sms &&
+                     (bpe + sms - 1) / sms * 32 <= kQMaxPiece;
+  static_assert(kQHeader + kQBufs * kQMaxPiece <= 232448, "shared memory budget of the single-pass quantiser");
+  err = cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * (size_t)(fused ? E + 3 : E), st);
+  if (err != cudaSuccess) return err;
+  if (fused) {
+    static int configured_dev = -1;
+    const int smem = kQHeader + kQBufs * kQMaxPiece;
+    if (configured_dev != dev) {
+      err = cudaFuncSetAttribute(quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (err != cudaSuccess) return err;
+      configured_dev = dev;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sms);
+    cfg.blockDim = dim3(kQThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the arrival waits end
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quantize_fused_kernel, w, (int)E, bpe, amax_ws, q, s, g, status);
+  }
   int gx = (int)((per / 8 + 255) / 256);
   if (gx > 64) gx = 64;
   amax_kernel<<<dim3(gx, (unsigned)E), 256, 0, st>>>(w, per, amax_ws);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const int64_t bpe = per / 16, nb = E * bpe;
+  const int64_t nb = E * bpe;
   encode_kernel<<<(unsigned)((nb + 255) / 256), 256, 0, st>>>(w, bpe, nb, amax_ws, q, s, g);
   return cudaGetLastError();
 }

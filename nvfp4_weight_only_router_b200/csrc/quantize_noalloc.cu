@@ -9,7 +9,9 @@
 // library routine; the caller still passes the input and output buffers.
 //
 // The array is shared by every call on a device and keeps the last call's
-// contents; each call clears the words it uses before the amax pass.  Calls
+// contents; each call clears the words it uses (one amax word per tensor,
+// plus three arrival counters when the tensors take the single-pass kernel)
+// before it reads them.  Calls
 // that overlap on the GPU race on the array.  Every GPU that loads the
 // library holds the array (16 KiB) until the process exits.
 #include <mutex>
@@ -58,8 +60,9 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* w, int64_t E, int64_t
   if (!aligned16(w) || !aligned16(q) || !aligned16(s) || !aligned16(g)) return NVFP4_ERR_ALIGNMENT;
   uint32_t* scratch = noalloc_scratch();
   if (!scratch) return NVFP4_ERR_CUDA;
-  // launch_quantize clears scratch[0..E) before the amax pass
+  // launch_quantize clears the scratch words it uses before the amax pass
   const cudaError_t e = nvfp4moe::launch_quantize(static_cast<const uint16_t*>(w), E, N, K, q, s, g,
-                                                  scratch, static_cast<cudaStream_t>(stream));
+                                                  scratch, kNoAllocMaxTensors, nvfp4moe::device_status_ptr(),
+                                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }

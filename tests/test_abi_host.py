@@ -54,7 +54,7 @@ def _experts(capi, E=128, H=2816, I=704, ptr=4096):
 
 def test_quantize_validation(capi):
     c = capi
-    assert c.nvfp4_quantize_workspace_bytes(128, 1408, 2816) == 512
+    assert c.nvfp4_quantize_workspace_bytes(128, 1408, 2816) == 768
     assert c.nvfp4_quantize_workspace_bytes(0, 1, 32) == 0
     P = 4096
     assert c.nvfp4_quantize(None, 1, 16, 32, P, P, P, P, 256, None) == c.NVFP4_ERR_INVALID_ARG

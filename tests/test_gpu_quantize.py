@@ -41,9 +41,24 @@ def test_random_shapes(dev, shape):
     _assert_equal_quant(_run(bits, dev), Q.quantize(bits))
 
 
-def test_edge_values(dev):
+def test_worked_example_rows_single_pass(dev):
+    """The worked example's blocks (ties at every E2M1 threshold, saturation,
+    zero and subnormal-scale blocks) repeated over enough rows that the
+    single-pass kernel (pieces of every tensor split over all CTAs) runs."""
+    rows = golden_lines("nvfp4_worked_example.txt")
+    w = np.array([float.fromhex(r[0]) for r in rows if r[0] not in ("G", "block")], np.float32)
+    row = np.concatenate([gen.bf16_bits(w), np.zeros(16, np.uint16)])
+    bits = np.tile(row[None, None, :], (2, 600, 1))
+    bits[1, 7] = 0x8000                      # one negative-zero row in the second tensor
+    _assert_equal_quant(_run(bits, dev), Q.quantize(bits))
+
+
+@pytest.mark.parametrize("N,K", [(8, 64), (16, 2816)])
+def test_edge_values(dev, N, K):
+    """Edge values through the two-pass kernels ([4, 8, 64]) and through the
+    single-pass kernel ([4, 16, 2816])."""
     rng = np.random.default_rng(12)
-    w = rng.standard_normal((4, 8, 64)).astype(np.float32)
+    w = rng.standard_normal((4, N, K)).astype(np.float32)
     w[0] = 0.0                              # all-zero tensor -> G = 0
     w[1, 0, :16] = 0.0                      # zero block
     w[1, 1, :16] = -0.0                     # negative-zero block
