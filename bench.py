@@ -38,9 +38,10 @@ ROUTER_BYTES = 128 * 2816 * 2 + 2816 * 2 + 128 * 2       # 726,784 (bf16 proj, s
 FLUSH_BYTES = 256 << 20
 
 # DRAM read + write per launch of the dominant kernel, from the ncu captures
-# summarised in profiles/ (stream_gemv_decode64.md, tc_moe_prefill4096.md);
+# summarised in profiles/ (stream_gemv_decode64.md, tc_moe_prefill4096.md,
+# quantize_fused_quantize.md);
 # None where no capture of the current kernel exists
-TRAFFIC_BYTES = {"decode64": 287.66e6, "prefill4096": 515.49e6}
+TRAFFIC_BYTES = {"decode64": 287.66e6, "prefill4096": 515.49e6, "quantize": 1278.80e6}
 
 WORKLOADS = {
     "decode64": {"T": 64, "layers": 1, "zipf": False,
@@ -391,7 +392,7 @@ def run_ours(args, wl, rank, world, local_rank):
         unit = "GB/s"
         roof = {"bound": "hbm", "kernel": "quantize_fused_kernel (single pass: amax + encode)",
                 "achieved": algo_bytes / (ms_per_step / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                "traffic": None, "peak_kind": peak_kind}
+                "traffic": TRAFFIC_BYTES.get(args.workload), "peak_kind": peak_kind}
         roof["frac"] = roof["achieved"] / roof["peak"]
         dtype = "u8"
         e2e = {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
