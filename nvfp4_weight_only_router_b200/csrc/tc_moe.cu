@@ -19,8 +19,9 @@
 // shuffle between adjacent lanes.
 //
 // Warp roles (16 warps): 0 TMA producer (activation box, packed-code boxes),
-// 1-3 MMA issuers (one thread each; from 64 tokens on two or three split the
-// tile's tokens), 4-7 epilogue (tensor memory -> registers -> global), 8-15
+// 1-3 MMA issuers (the whole warp runs the loop so the MMA operands stay
+// warp-uniform, one elected lane issues; from 64 tokens on two or three split
+// the tile's tokens), 4-7 epilogue (tensor memory -> registers -> global), 8-15
 // dequantisation (warp w owns tensor-memory lanes 32(w%4).. and K half
 // (w-8)/4; it reads its row's e4m3 scales from global memory three chunks
 // ahead, so the shared memory goes to a deeper load ring).
@@ -147,6 +148,28 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
+// Issued by the whole (converged) warp, performed by one elected lane: the
+// operands are computed by every lane alike, so they stay warp-uniform.
+__device__ __forceinline__ void tc_mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+// The commit of the same elected lane (elect.sync in a converged warp picks
+// the same lane every time, so it covers that lane's MMAs).
+__device__ __forceinline__ void tc_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 
@@ -305,7 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpMma && warp < kWarpMma + C::NI) {
     // ---------------------------------------------------------- MMA issuers
-    if (lane == 0) {
+    // The whole warp runs the loop (so descriptors and addresses are
+    // warp-uniform); one elected lane issues each MMA and commit.
+    {
       const int hh = warp - kWarpMma;  // token share of this issuer
       uint32_t kiter = 0, titer = 0;
       bool ok = true;
@@ -318,17 +343,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int mine = min(C::NH, min(NT, ti.cnt - ti.i * NT) - hh * C::NH);
         const int nmma = mine <= 0 ? 0 : ((mine + 15) & ~15);
         const uint32_t idesc = make_idesc_f16(kRows, nmma > 0 ? nmma : 16);
-        if (duse > 0 && !wait_or_abort(sm, &sm.d_empty[db], (duse - 1) & 1, p.status)) break;
+        if (duse > 0) ok = wait_or_abort(sm, &sm.d_empty[db], (duse - 1) & 1, p.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);  // one decision for the warp
+        if (!ok) break;
         tc_fence_after();
         const uint32_t d = taddr + (uint32_t)(db * C::NACC * NT + hh * C::NH);
         for (int kc = 0; kc < C::KC; ++kc, ++kiter) {
           const int s = kiter % C::NS, use = kiter / C::NS;
           const int a = kiter % C::NA, ause = kiter / C::NA;
-          if (!wait_or_abort(sm, &sm.full[s], use & 1, p.status) ||
-              !wait_or_abort(sm, &sm.a_full[a], ause & 1, p.status)) {
-            ok = false;
-            break;
-          }
+          ok = wait_or_abort(sm, &sm.full[s], use & 1, p.status) && wait_or_abort(sm, &sm.a_full[a], ause & 1, p.status);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
           tc_fence_after();
           // rows hh*NH.. of the 128B-swizzled activation tile (NH*128 bytes = whole 8-row atoms)
           const uint64_t bd = make_sw128_desc(smem_u32(sm.x[s]) + (uint32_t)(hh * C::NH * 128));
@@ -336,16 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (nmma > 0) {
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk)
-              tc_mma_ts(d + (uint32_t)((kk % C::NACC) * NT), a0 + (uint32_t)(kk * 8), bd + (uint64_t)(kk * 2), idesc,
-                        kc != 0 || kk >= C::NACC);
+              tc_mma_ts_warp(d + (uint32_t)((kk % C::NACC) * NT), a0 + (uint32_t)(kk * 8), bd + (uint64_t)(kk * 2),
+                             idesc, kc != 0 || kk >= C::NACC);
           }
-          tc_commit(&sm.empty[s]);  // with no MMA in flight the arrival is immediate
+          tc_commit_warp(&sm.empty[s]);  // with no MMA in flight the arrival is immediate
         }
         if (!ok) break;
-        tc_commit(&sm.d_full[db]);
+        tc_commit_warp(&sm.d_full[db]);
       }
-      tc_commit(&sm.fin);
+      tc_commit_warp(&sm.fin);
       mbar_wait_bounded(&sm.fin, 0);
+      __syncwarp();
     }
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     // ------------------------------------------------------------ epilogue
