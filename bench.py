@@ -189,6 +189,30 @@ def run_reference(args, wl, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------ replica aggregation
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest `value` over all ranks (every rank gets it): step times
+    are reported as the slowest replica's."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: the units all replicas processed over `steps`
+    steps, divided by the (slowest replica's) time."""
+    return world * units_per_rank * steps / (total_ms / 1e3)
+
+
+def replica_x_seed(rank: int, n_pool: int, i: int) -> int:
+    """Seed of input i of a replica's pool: disjoint pools across ranks."""
+    return 10_000 + rank * n_pool + i
+
+
 # ----------------------------------------------------------------- ours
 def run_ours(args, wl, rank, world, local_rank):
     import torch
@@ -242,7 +266,7 @@ def run_ours(args, wl, rank, world, local_rank):
             layers.append(lib.MoeLayer(lib.Experts.from_host(ex, dev), lib.Router.from_host(rt, dev),
                                        max_tokens=T))
             del ex
-        xs_host = np.stack([gen.make_x(10_000 + rank * n_pool + i, T) for i in range(n_pool)])
+        xs_host = np.stack([gen.make_x(replica_x_seed(rank, n_pool, i), T) for i in range(n_pool)])
         x_pool = bf(xs_host).to(dev)
         x_pin = bf(xs_host).pin_memory()
         xs = torch.empty((T, 2816), dtype=torch.bfloat16, device=dev)
@@ -357,11 +381,7 @@ def run_ours(args, wl, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop()
 
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
 
     # -------- e2e through the public API with host buffers
@@ -378,17 +398,13 @@ def run_ours(args, wl, rank, world, local_rank):
             end.record()
             end.synchronize()
             e_ms.append(start.elapsed_time(end))
-        e_tot = sum(e_ms)
-        if world > 1:
-            t = torch.tensor([e_tot], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_tot = float(t.item())
-        e2e = {"value": world * T * args.steps / (e_tot / 1e3), "unit": "tokens/s",
+        e_tot = max_over_ranks(sum(e_ms), world, dev)
+        e2e = {"value": job_rate(T, world, args.steps, e_tot), "unit": "tokens/s",
                "h2d_bytes_per_step": T * 2816 * 2, "d2h_bytes_per_step": T * 2816 * 2}
 
     # -------- roofline of the dominant kernel
     if args.workload == "quantize":
-        value = world * algo_bytes * args.steps / (total_ms / 1e3) / 1e9
+        value = job_rate(algo_bytes, world, args.steps, total_ms) / 1e9
         unit = "GB/s"
         roof = {"bound": "hbm", "kernel": "quantize_fused_kernel (single pass: amax + encode)",
                 "achieved": algo_bytes / (ms_per_step / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
@@ -398,7 +414,7 @@ def run_ours(args, wl, rank, world, local_rank):
         e2e = {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
                "note": "weights resident; no host copies in a quantise step"}
     else:
-        value = world * T * args.steps / (total_ms / 1e3)
+        value = job_rate(T, world, args.steps, total_ms)
         unit = "tokens/s"
         ph = np.array(phase_ms)  # [steps, 5]: route, permute, gate_up, down, combine
         n_act = np.array(act_counts, np.float64)
