@@ -112,7 +112,14 @@ typedef struct {
  *   s_dev  u8 [E, N, K/16] (out)    g_dev f32 [E] (out)
  * Requires E >= 1, N >= 1, K >= 16, K % 32 == 0, N * K < 2^31.  NaN/Inf
  * inputs are not supported (their codes are unspecified).
- * Workspace: nvfp4_quantize_workspace_bytes(E, N, K) bytes, 256-aligned.
+ * Workspace: nvfp4_quantize_workspace_bytes(E, N, K) bytes, 256-aligned
+ * (E amax words and three arrival counters; the call clears what it uses).
+ * Execution: when one tensor's share per SM fits on chip (N * K / 16 blocks
+ * of 32 bytes split over all SMs, at most 54 KB each, and at least 8 blocks
+ * per SM) the call is one cooperative launch of one CTA per SM that reads
+ * every weight once; it occupies the whole GPU while it runs and returns
+ * NVFP4_ERR_CUDA if the CTAs cannot all be resident.  Other shapes take two
+ * passes (amax, then encode).  Both give the same bytes.
  * ------------------------------------------------------------------------- */
 NVFP4MOE_API size_t nvfp4_quantize_workspace_bytes(int64_t E, int64_t N, int64_t K);
 NVFP4MOE_API nvfp4_status nvfp4_quantize(const void* w_dev, int64_t E, int64_t N, int64_t K,
