@@ -117,9 +117,10 @@ typedef struct {
  * Execution: when one tensor's share per SM fits on chip (N * K / 16 blocks
  * of 32 bytes split over all SMs, at most 54 KB each, and at least 8 blocks
  * per SM) the call is one cooperative launch of one CTA per SM that reads
- * every weight once; it occupies the whole GPU while it runs and returns
- * NVFP4_ERR_CUDA if the CTAs cannot all be resident.  Other shapes take two
- * passes (amax, then encode).  Both give the same bytes.
+ * every weight once; it occupies the whole GPU while it runs (if the
+ * context cannot hold one CTA on every SM at once, the call takes the two
+ * passes instead).  Other shapes take two passes (amax, then encode).  Both
+ * give the same bytes.
  * ------------------------------------------------------------------------- */
 NVFP4MOE_API size_t nvfp4_quantize_workspace_bytes(int64_t E, int64_t N, int64_t K);
 NVFP4MOE_API nvfp4_status nvfp4_quantize(const void* w_dev, int64_t E, int64_t N, int64_t K,

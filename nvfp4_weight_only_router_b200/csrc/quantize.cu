@@ -467,7 +467,11 @@ cudaError_t launch_quantize(const uint16_t* w, int64_t E, int64_t N, int64_t K, 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quantize_fused_kernel, w, (int)E, bpe, amax_ws, q, s, g, status);
+    err = cudaLaunchKernelEx(&cfg, quantize_fused_kernel, w, (int)E, bpe, amax_ws, q, s, g, status);
+    // not every SM available to this context (a partitioned GPU): the two
+    // passes below need no co-residency (their amax words are cleared too)
+    if (err != cudaErrorCooperativeLaunchTooLarge) return err;
+    (void)cudaGetLastError();
   }
   int gx = (int)((per / 8 + 255) / 256);
   if (gx > 64) gx = 64;
