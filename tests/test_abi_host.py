@@ -65,6 +65,11 @@ def test_quantize_validation(capi):
     assert c.nvfp4_quantize(P, 1, 16, 32, P, P, P, P, 0, None) == c.NVFP4_ERR_WORKSPACE
     assert c.nvfp4_quantize(P, 1, 16, 32, P, P, P, P + 16, 4096, None) == c.NVFP4_ERR_ALIGNMENT
     assert c.nvfp4_quantize(P, 1, 1 << 20, 4096, P, P, P, P, 4096, None) == c.NVFP4_ERR_UNSUPPORTED
+    # E amax words plus the single-pass kernel's three arrival counters
+    assert c.nvfp4_quantize_workspace_bytes(1, 16, 32) == 256
+    assert c.nvfp4_quantize_workspace_bytes(61, 16, 32) == 256
+    assert c.nvfp4_quantize_workspace_bytes(62, 16, 32) == 512
+    assert c.nvfp4_quantize(P, 128, 1408, 2816, P, P, P, P, 512, None) == c.NVFP4_ERR_WORKSPACE
 
 
 def test_route_validation(capi):
