@@ -6,7 +6,9 @@
 
 A step is one pass of the whole hot path -- route, permute, gate_up + GELU,
 down, combine -- over one batch of synthetic tokens (the default workload:
-one MoE layer of the Gemma-4-26B-A4B shapes, T=64 decode tokens).  Inputs are
+one MoE layer of the Gemma-4-26B-A4B shapes, T=64 decode tokens; the default
+run also times the T=4096 prefill workload on the same layer and reports it
+under "prefill", the metric's tensor-core half).  Inputs are
 resident in HBM before the timed region; L2 is flushed (256 MiB write)
 between timed steps, outside the timed events.  Each rank runs its own replica
 (the branch is per-token independent; no collective on the data path);
@@ -37,11 +39,32 @@ EXPERT_BYTES = GU_EXPERT_BYTES + DN_EXPERT_BYTES        # 3,345,416
 ROUTER_BYTES = 128 * 2816 * 2 + 2816 * 2 + 128 * 2       # 726,784 (bf16 proj, scale, pes)
 FLUSH_BYTES = 256 << 20
 
-# DRAM read + write per launch of the dominant kernel, from the ncu captures
-# summarised in profiles/ (stream_gemv_decode64.md, quantize_fused_quantize.md;
-# the prefill GEMM changed after tc_moe_prefill4096.md was captured);
-# None where no capture of the current kernel exists
-TRAFFIC_BYTES = {"decode64": 287.66e6, "prefill4096": None, "quantize": 1278.80e6}
+# DRAM read + write per launch of each workload's dominant kernel, as taken
+# by an ncu capture, with the SHA-256 of the kernel's source files at capture
+# time; a figure whose sources have changed since is reported as null.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def source_digest(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in sorted(paths):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(rel.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(workload: str):
+    """(bytes per launch, kernel) of the workload's dominant kernel from the
+    capture file, or (None, None) if absent or taken on other sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[workload]
+        if rec["sources_sha256"] != source_digest(rec["sources"]):
+            return None, rec.get("kernel")
+        return float(rec["dram_bytes_per_launch"]), rec.get("kernel")
+    except Exception:
+        return None, None
 
 WORKLOADS = {
     "decode64": {"T": 64, "layers": 1, "zipf": False,
@@ -214,34 +237,55 @@ def replica_x_seed(rank: int, n_pool: int, i: int) -> int:
 
 
 # ----------------------------------------------------------------- ours
-def run_ours(args, wl, rank, world, local_rank):
+class _Ctx:
+    """Per-process state shared by the measured workloads."""
+
+    def __init__(self, rank, world, local_rank):
+        import torch
+        self.rank, self.world, self.local_rank = rank, world, local_rank
+        self.dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(self.dev)
+        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=self.dev)
+        self.hbm_peak, self.tc_peak, self.tc_peak_sus, self.peak_kind = measured_peaks()
+        self._experts = {}
+
+    def experts(self, seed):
+        """Device copy of a layer's experts (shared by workloads on the same seed)."""
+        import moe_inputs as gen
+        import nvfp4_weight_only_router_b200 as lib
+        if seed not in self._experts:
+            ex = gen.make_experts(seed)
+            self._experts[seed] = lib.Experts.from_host(ex, self.dev)
+            del ex
+        return self._experts[seed]
+
+
+def _bf(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+def measure(ctx, workload, args, cpu_baseline=True):
+    """Time one workload: W warm-up steps (and at least --min-warmup-s of
+    load), then exactly K timed steps between L2 flushes, CUDA events on the
+    launching stream, max over ranks.  Returns the JSON-line fields."""
+    import ctypes
     import torch
     import torch.distributed as dist
     import moe_inputs as gen
     import nvfp4_weight_only_router_b200 as lib
-    from nvfp4_weight_only_router_b200 import build as bld
+    from nvfp4_weight_only_router_b200 import capi
 
-    if rank == 0 or world == 1:
-        bld.build()
-    if world > 1:
-        dist.barrier()
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    hbm_peak, tc_peak, tc_peak_sus, peak_kind = measured_peaks()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def bf(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
-
+    wl = WORKLOADS[workload]
+    rank, world, dev = ctx.rank, ctx.world, ctx.dev
     T = wl["T"]
     n_pool = 64
     extra = {}
     events = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-    ev_ptrs = None
 
-    if args.workload == "quantize":
+    if workload == "quantize":
         w = gen.make_quant_weights(4, 128, 1408, 2816)
-        w_pin = bf(w).pin_memory()  # host copy of the weights for the end-to-end pass
+        w_pin = _bf(w).pin_memory()  # host copy of the weights for the end-to-end pass
         wd = w_pin.to(dev)
         del w
         q = torch.empty((128, 1408, 1408), dtype=torch.uint8, device=dev)
@@ -250,7 +294,6 @@ def run_ours(args, wl, rank, world, local_rank):
         q_pin = torch.empty(q.shape, dtype=torch.uint8).pin_memory()
         s_pin = torch.empty(s.shape, dtype=torch.uint8).pin_memory()
         g_pin = torch.empty(g.shape, dtype=torch.float32).pin_memory()
-        from nvfp4_weight_only_router_b200 import capi
         ws_bytes = capi.nvfp4_quantize_workspace_bytes(128, 1408, 2816)
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
@@ -258,21 +301,21 @@ def run_ours(args, wl, rank, world, local_rank):
             capi.check(capi.nvfp4_quantize(wd.data_ptr(), 128, 1408, 2816, q.data_ptr(), s.data_ptr(),
                                            g.data_ptr(), ws.data_ptr(), ws_bytes,
                                            torch.cuda.current_stream().cuda_stream))
+
+        def prepare(i):
+            pass
         algo_bytes = wd.numel() * 2 + q.numel() + s.numel() + 128 * 4
         kernels_per_step = 1  # the single-pass kernel (the clearing of its counters is a memset)
     else:
         layers = []
         seeds = [0] if wl["layers"] == 1 else gen.layer_seed_plan(wl["layers"])
-        for li, sd in enumerate(seeds):
-            ex = gen.make_experts(sd)
+        for sd in seeds:
             rt = gen.make_router(1 if wl["layers"] == 1 else 1000 + sd,
                                  bias=gen.zipf_bias(7) if wl["zipf"] else None)
-            layers.append(lib.MoeLayer(lib.Experts.from_host(ex, dev), lib.Router.from_host(rt, dev),
-                                       max_tokens=T))
-            del ex
+            layers.append(lib.MoeLayer(ctx.experts(sd), lib.Router.from_host(rt, dev), max_tokens=T))
         xs_host = np.stack([gen.make_x(replica_x_seed(rank, n_pool, i), T) for i in range(n_pool)])
-        x_pool = bf(xs_host).to(dev)
-        x_pin = bf(xs_host).pin_memory()
+        x_pool = _bf(xs_host).to(dev)
+        x_pin = _bf(xs_host).pin_memory()
         xs = torch.empty((T, 2816), dtype=torch.bfloat16, device=dev)
         y = torch.empty_like(xs)
         y_pin = torch.empty((T, 2816), dtype=torch.bfloat16).pin_memory()
@@ -280,8 +323,6 @@ def run_ours(args, wl, rank, world, local_rank):
         xn = torch.empty_like(xs)
 
         def fwd_layer(layer, xin, yout, profiled):
-            from nvfp4_weight_only_router_b200 import capi
-            import ctypes
             st = torch.cuda.current_stream().cuda_stream
             if profiled:
                 arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
@@ -337,13 +378,12 @@ def run_ours(args, wl, rank, world, local_rank):
         per_layer = 5 if T * 8 <= 1024 else 7
         kernels_per_step = per_layer * len(layers) + (len(layers) + 1 if len(layers) > 1 else 0)
 
-    # -------- warm-up (at least W steps and at least 1 s, so the clock sampler sees load)
-    sampler = ClockSampler(physical_gpu_index(local_rank))
+    # -------- warm-up (at least W steps and at least --min-warmup-s, so the clock sampler sees load)
+    sampler = ClockSampler(physical_gpu_index(ctx.local_rank))
     t_end = time.perf_counter() + args.min_warmup_s
     i = 0
     while i < args.warmup or time.perf_counter() < t_end:
-        if args.workload != "quantize":
-            prepare(i)
+        prepare(i)
         step(i)
         i += 1
     torch.cuda.synchronize()
@@ -355,24 +395,23 @@ def run_ours(args, wl, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     for k in range(args.steps):
-        flush.zero_()
-        if args.workload != "quantize":
-            prepare(k)
+        ctx.flush.zero_()
+        prepare(k)
         start.record()
         step(k)
         end.record()
         torch.cuda.synchronize()
         step_ms.append(start.elapsed_time(end))
-        if args.workload != "quantize":
+        if workload != "quantize":
             act_counts.append(int((layers[0].views(T)["counts"] > 0).sum().item()))
     torch.cuda.synchronize()
     # phase breakdown (and the dominant kernel's duration for the roofline):
     # the same K steps again, each replaying the graph whose event-record
     # nodes sit between the phases, on the launching stream
     prof_ms = []
-    if args.workload != "quantize":
+    if workload != "quantize":
         for k in range(args.steps):
-            flush.zero_()
+            ctx.flush.zero_()
             prepare(k)
             start.record()
             step_prof(k)
@@ -389,13 +428,12 @@ def run_ours(args, wl, rank, world, local_rank):
     ms_per_step = total_ms / args.steps
 
     # -------- e2e through the public API with host buffers
-    e2e = None
-    if args.workload == "quantize":
+    if workload == "quantize":
         # the weights come from pinned host memory and the codes, scales and
         # global scales go back to it, every step
         e_ms = []
         for k in range(args.steps):
-            flush.zero_()
+            ctx.flush.zero_()
             torch.cuda.synchronize()
             start.record()
             wd.copy_(w_pin, non_blocking=True)
@@ -413,7 +451,7 @@ def run_ours(args, wl, rank, world, local_rank):
     else:
         e_ms = []
         for k in range(args.steps):
-            flush.zero_()
+            ctx.flush.zero_()
             torch.cuda.synchronize()
             start.record()
             xs.copy_(x_pin[k % n_pool], non_blocking=True)
@@ -427,12 +465,13 @@ def run_ours(args, wl, rank, world, local_rank):
                "h2d_bytes_per_step": T * 2816 * 2, "d2h_bytes_per_step": T * 2816 * 2}
 
     # -------- roofline of the dominant kernel
-    if args.workload == "quantize":
+    traffic, traffic_kernel = captured_traffic(workload)
+    if workload == "quantize":
         value = job_rate(algo_bytes, world, args.steps, total_ms) / 1e9
         unit = "GB/s"
         roof = {"bound": "hbm", "kernel": "quantize_fused_kernel (single pass: amax + encode)",
-                "achieved": algo_bytes / (ms_per_step / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                "traffic": TRAFFIC_BYTES.get(args.workload), "peak_kind": peak_kind}
+                "achieved": algo_bytes / (ms_per_step / 1e3) / 1e9, "peak": ctx.hbm_peak, "unit": "GB/s",
+                "traffic": traffic, "peak_kind": ctx.peak_kind, "algorithmic_per_launch": float(algo_bytes)}
         roof["frac"] = roof["achieved"] / roof["peak"]
         dtype = "u8"
     else:
@@ -445,16 +484,16 @@ def run_ours(args, wl, rank, world, local_rank):
         gu_flops = 2.0 * S * 1408 * 2816
         gu_ms = ph[:, 2]
         if T >= 1024:
+            # a sub-millisecond kernel timed between L2 flushes: the burst peak
             ach = gu_flops / (gu_ms.mean() / 1e3) / 1e12
-            roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM + GELU", "achieved": ach,
-                    "peak": tc_peak_sus, "unit": "TFLOP/s", "traffic": TRAFFIC_BYTES.get(args.workload),
-                    "peak_kind": peak_kind + " sustained",
-                    "algorithmic_per_launch": gu_flops}
+            roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM + GELU (tcgen05)", "achieved": ach,
+                    "peak": ctx.tc_peak, "unit": "TFLOP/s", "traffic": traffic,
+                    "peak_kind": ctx.peak_kind + " burst bf16", "algorithmic_per_launch": gu_flops}
         else:
             ach = gu_bytes.sum() / (gu_ms.sum() / 1e3) / 1e9
             roof = {"bound": "hbm", "kernel": "gate_up grouped GEMV + GELU", "achieved": ach,
-                    "peak": hbm_peak, "unit": "GB/s", "traffic": TRAFFIC_BYTES.get(args.workload),
-                    "peak_kind": peak_kind,
+                    "peak": ctx.hbm_peak, "unit": "GB/s", "traffic": traffic,
+                    "peak_kind": ctx.peak_kind,
                     "algorithmic_per_launch": float(gu_bytes.mean())}
         roof["frac"] = roof["achieved"] / roof["peak"]
         step_bytes = n_act * EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2
@@ -468,34 +507,56 @@ def run_ours(args, wl, rank, world, local_rank):
             "layer_tflops": float(2.0 * S * (1408 * 2816 + 2816 * 704) * wl["layers"] / (ms_per_step / 1e3) / 1e12),
         }
         dtype = "f16xe2m1"
+    if traffic_kernel:
+        roof["traffic_kernel"] = traffic_kernel
 
     cpu = None
-    if rank == 0 and not args.no_cpu_baseline:
-        tokens = 2 if args.workload != "prefill4096" else 4
-        sample = OracleSample(args.workload, wl, tokens)
+    if rank == 0 and cpu_baseline:
+        tokens = 2 if workload != "prefill4096" else 4
+        sample = OracleSample(workload, wl, tokens)
         v, u, dt = sample.run()
         what = sample.what
-        if args.workload == "stack30":
+        if workload == "stack30":
             v /= 30.0
             what += " (value per 30-layer step)"
         cpu = {"value": v, "unit": u, "cores": blas_threads(), "kind": "oracle",
                "sample": what + f" ({dt:.1f} s)"}
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
-            "config": {"workload": args.workload, "desc": wl["desc"], "T": T,
-                       "l2": "256 MiB flush write between timed steps",
-                       "graph": args.workload != "quantize", "parallelism": f"replicas x{world}"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": kernels_per_step * args.steps, "clocks": clocks,
-        }
-        line.update(extra)
-        print(json.dumps(line), flush=True)
-    if args.workload != "quantize":
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {"workload": workload, "desc": wl["desc"], "T": T,
+                   "l2": "256 MiB flush write between timed steps",
+                   "graph": workload != "quantize", "parallelism": f"replicas x{world}"},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": kernels_per_step * args.steps, "clocks": clocks,
+    }
+    line.update(extra)
+    if workload != "quantize":
         del graph, graph_prof
+    return line
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch.distributed as dist
+    from nvfp4_weight_only_router_b200 import build as bld
+
+    if rank == 0 or world == 1:
+        bld.build()
+    if world > 1:
+        dist.barrier()
+    ctx = _Ctx(rank, world, local_rank)
+    line = measure(ctx, args.workload, args, cpu_baseline=not args.no_cpu_baseline)
+    if args.workload == "decode64" and not args.no_prefill:
+        # the metric's other half: the prefill workload on the same experts, in
+        # the same invocation (its own warm-up, timed steps and clock record)
+        p = measure(ctx, "prefill4096", args, cpu_baseline=False)
+        line["prefill"] = {k: p[k] for k in ("value", "unit", "ms_per_step", "roofline", "clocks", "e2e",
+                                             "gpu_launches", "phase_ms_mean", "layer_tflops")}
+        line["prefill"]["config"] = p["config"]
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def main():
@@ -506,6 +567,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode64", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="decode64 only: skip the prefill4096 half of the metric")
     ap.add_argument("--min-warmup-s", type=float, default=1.0,
                     help="keep warming up for at least this long (the clock sampler needs load)")
     args = ap.parse_args()
@@ -525,7 +588,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, wl, rank, world, local_rank)
+        run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

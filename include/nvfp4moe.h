@@ -23,8 +23,9 @@
  *     invalid call returns an error status and enqueues nothing.
  *   - Every device pointer must be 16-byte aligned (NVFP4_ERR_ALIGNMENT
  *     otherwise) and workspaces 256-byte aligned.
- *   - Errors are returned, never thrown or printed.  A CUDA launch error is
- *     reported as NVFP4_ERR_CUDA; details via cudaGetLastError.
+ *   - Errors are returned, never thrown or printed.  A failed CUDA runtime
+ *     call or launch is reported as NVFP4_ERR_CUDA; nvfp4_last_cuda_error
+ *     gives the CUDA error behind it.
  *   - Calls that share a workspace must not overlap on the GPU.
  *
  * Tensor layouts (row-major, innermost last)
@@ -51,7 +52,7 @@
 extern "C" {
 #endif
 
-#define NVFP4MOE_ABI_VERSION 1
+#define NVFP4MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define NVFP4MOE_API __attribute__((visibility("default")))
@@ -67,7 +68,9 @@ typedef enum {
   NVFP4_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
   NVFP4_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (device status) */
   NVFP4_ERR_UNSUPPORTED = 6,   /* valid but not implemented shape (see each call) */
-  NVFP4_ERR_DEVICE = 7         /* a kernel detected bad input data (device status) */
+  NVFP4_ERR_DEVICE = 7,        /* a kernel detected bad input data (device status) */
+  NVFP4_ERR_RANGE = 8          /* an activation left the f16 operand range and was
+                                  saturated (device status; see moe_nvfp4_forward) */
 } nvfp4_status;
 
 /* Router parameters ("Gemma 4 26B-A4B (MoE) - Core AI", router description
@@ -78,7 +81,7 @@ typedef struct {
   const void* per_expert_scale;  /* bf16 [E] */
   const float* logit_bias;       /* f32 [E], added to the logits; NULL = none */
   int32_t E;                     /* number of experts: must be 128 */
-  int32_t H;                     /* hidden size: multiple of 128, <= 16384 */
+  int32_t H;                     /* hidden size: a multiple of 256 in [2048, 4096] */
   int32_t top_k;                 /* must be 8 */
   float eps;                     /* RMSNorm epsilon (the pages are silent; 1e-6) */
 } moe_router;
@@ -139,7 +142,11 @@ NVFP4MOE_API nvfp4_status nvfp4_quantize(const void* w_dev, int64_t E, int64_t N
  * Same arguments, layouts, results and limits as nvfp4_quantize, plus
  * E <= 4096 (NVFP4_ERR_UNSUPPORTED beyond).  The first call on a device looks
  * up the array's device address (cudaGetSymbolAddress, with that device
- * current); make that first call before any stream capture.  All calls on a
+ * current); make that first call before any stream capture.  With CUDA's
+ * default lazy module loading, that first call on each device (or loading the
+ * library, with CUDA_MODULE_LOADING=EAGER) is also when the driver places the
+ * array and the library's code on the device: callers with a strict
+ * no-allocation window make one call before the window opens.  All calls on a
  * device share the array, which keeps the last call's contents (each call
  * clears what it needs): calls that overlap on the GPU race. */
 NVFP4MOE_API nvfp4_status nvfp4_quantize_noalloc(const void* w_dev, int64_t E, int64_t N, int64_t K,
@@ -163,8 +170,10 @@ NVFP4MOE_API nvfp4_status nvfp4_dequantize(const uint8_t* q_dev, const uint8_t* 
  *   ids_dev  int32 [T, top_k] (out), by descending p; the selection compares
  *            the fp32 logits (softmax is monotone), equal logits -> lower id first
  *   w_dev    f32 [T, top_k] (out)
- * Requires 1 <= T <= 65536, E == 128, top_k == 8, H % 128 == 0, H <= 16384.
- * Workspace: moe_route_workspace_bytes(T, router) bytes.
+ * Requires 1 <= T <= 65536, E == 128, top_k == 8, H % 256 == 0 and
+ * 2048 <= H <= 4096 (NVFP4_ERR_UNSUPPORTED otherwise).
+ * Workspace: moe_route_workspace_bytes(T, router) bytes (the kernels keep
+ * their scratch on chip; the query returns 256).
  * ------------------------------------------------------------------------- */
 NVFP4MOE_API size_t moe_route_workspace_bytes(int32_t T, const moe_router* router);
 NVFP4MOE_API nvfp4_status moe_route(const void* x_dev, int32_t T, const moe_router* router,
@@ -180,8 +189,16 @@ NVFP4MOE_API nvfp4_status moe_route(const void* x_dev, int32_t T, const moe_rout
  *   h    = gelu_tanh(gate) * up
  *   out  = G_d[e] * (Wq_down[e] h)
  * where Wq = e2m1 * e4m3 is exact in f16.  x and h enter the tensor cores as
- * f16 (x converted with saturation to +-65504; h rounded to f16), products are
- * accumulated in fp32, the combine is fp32, y is rounded once to bf16.
+ * f16 under an exact power-of-two prescale per token: with e_t = floor(log2
+ * max|x_t|), x_t enters as x_t * 2^(15 - e_t) (every bf16 element down to
+ * 2^-32 of the row maximum is exact) and h as h * 2^(-2 e_t) rounded to f16
+ * (h grows as x^2, so its f16 precision does not depend on the size of x);
+ * the fp32 epilogues undo both scalings.  Products are accumulated in fp32,
+ * the combine is fp32, y is rounded once to bf16.  A row maximum outside
+ * [2^-111, 2^113), or a scaled h beyond the f16 range (|h| >= 65520 *
+ * 2^(2 e_t): weights whose gated outputs exceed ~65000 for an input of unit
+ * maximum), saturates and records NVFP4_ERR_RANGE in the device status.
+ * x must be finite.
  *   x_dev bf16 [T, H] (in), y_dev bf16 [T, H] (out)
  * Requires 1 <= T <= 65536, E == 128, H == 2816, I == 704, top_k == 8.
  * Workspace: moe_forward_workspace_bytes(T, experts, router) bytes.
@@ -209,12 +226,36 @@ NVFP4MOE_API nvfp4_status moe_nvfp4_forward_profiled(const void* x_dev, int32_t 
  *   counts int32 [E], offsets int32 [E+1] (exclusive prefix of counts),
  *   sorted_slot int32 [T*8] (slots t*8+j grouped by expert, stable),
  *   slot_pos int32 [T*8] (inverse permutation),
- *   h f16 [T*8, I] (gated hidden, rows in sorted_slot order). */
+ *   xexp int32 [T*8] (e_t of each sorted slot's token: the prescale exponent),
+ *   h f16 [T*8, I] (gated hidden, rows in sorted_slot order, row p holding
+ *     h * 2^(-2 e) with e = xexp[p] clamped to [-63, 63]). */
 typedef struct {
-  size_t ids, weights, counts, offsets, sorted_slot, slot_pos, h;
+  size_t ids, weights, counts, offsets, sorted_slot, slot_pos, xexp, h;
 } moe_forward_views;
 NVFP4MOE_API nvfp4_status moe_forward_workspace_views(int32_t T, const moe_experts* experts,
                                          const moe_router* router, moe_forward_views* out);
+
+/* ---------------------------------------------------------------------------
+ * moe_permute: the token permutation of moe_nvfp4_forward on its own -- the
+ * T*8 routing slots s = t*8 + j grouped by expert with a stable counting sort
+ * (the sort-by-expert step of the batched expert kernel, "Gemma 4 26B-A4B
+ * (MoE) - Core AI", "Decode only ...").
+ *   ids_dev         int32 [T, 8] (in), expert ids in [0, 128)
+ *   counts_dev      int32 [128] (out), slots per expert
+ *   offsets_dev     int32 [129] (out), exclusive prefix of counts
+ *   sorted_slot_dev int32 [T*8] (out), slots grouped by expert, increasing
+ *                   slot order within an expert
+ *   slot_pos_dev    int32 [T*8] (out), inverse: sorted_slot[slot_pos[s]] == s
+ * An id outside [0, 128) records NVFP4_ERR_DEVICE in the device status; that
+ * slot is left out of every expert (slot_pos -1, not counted) and the entries
+ * of sorted_slot past offsets[128] are unspecified.
+ * Requires 1 <= T <= 65536.  Workspace: moe_permute_workspace_bytes(T).
+ * ------------------------------------------------------------------------- */
+NVFP4MOE_API size_t moe_permute_workspace_bytes(int32_t T);
+NVFP4MOE_API nvfp4_status moe_permute(const int32_t* ids_dev, int32_t T, int32_t* counts_dev,
+                                      int32_t* offsets_dev, int32_t* sorted_slot_dev,
+                                      int32_t* slot_pos_dev, void* ws_dev, size_t ws_bytes,
+                                      void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_residual_rmsnorm: one link of a chained layer stack,
@@ -234,6 +275,22 @@ NVFP4MOE_API nvfp4_status moe_residual_rmsnorm(float* res_dev, const void* y_dev
  * error (NVFP4_OK if none) and clears the word.
  * ------------------------------------------------------------------------- */
 NVFP4MOE_API nvfp4_status nvfp4_get_device_status(void* stream);
+
+/* nvfp4_selftest_wait_timeout: exercises the device-side failure path of the
+ * bounded waits, so a deployment can check it on its driver without harming
+ * the GPU.  It runs nvfp4_quantize's single-pass kernel on the given tensors
+ * with a cross-CTA arrival count that can never be reached and every wait
+ * limited to limit_us microseconds: each CTA gives up, records
+ * NVFP4_ERR_TIMEOUT in the device status word, lets its own copies land and
+ * exits, so the context stays usable (the next nvfp4_get_device_status
+ * returns NVFP4_ERR_TIMEOUT).  The outputs are left unspecified.  Same
+ * arguments and limits as nvfp4_quantize plus 1 <= limit_us <= 1000000;
+ * NVFP4_ERR_UNSUPPORTED for a shape that does not take the single-pass
+ * kernel.  The pages have no counterpart of this entry point. */
+NVFP4MOE_API nvfp4_status nvfp4_selftest_wait_timeout(const void* w_dev, int64_t E, int64_t N, int64_t K,
+                                                      uint8_t* q_dev, uint8_t* s_dev, float* g_dev,
+                                                      void* ws_dev, size_t ws_bytes, uint32_t limit_us,
+                                                      void* stream);
 
 NVFP4MOE_API const char* nvfp4_status_string(nvfp4_status status);
 NVFP4MOE_API int nvfp4_abi_version(void);

@@ -5,8 +5,8 @@ Two layers:
   * the C ABI under its own names (`nvfp4_quantize`, `moe_route`,
     `moe_nvfp4_forward`, ... in `nvfp4_weight_only_router_b200.capi`): raw
     device pointers and sizes, returning the status code;
-  * torch conveniences (`quantize`, `dequantize`, `route`, `MoeLayer`,
-    `residual_rmsnorm`): they allocate outputs and workspaces with torch and
+  * torch conveniences (`quantize`, `dequantize`, `route`, `permute`,
+    `MoeLayer`, `residual_rmsnorm`): they allocate outputs and workspaces with torch and
     pass pointers to the same C calls on torch's current stream.
 
 Every computation runs in the library's CUDA kernels; there is no fallback.
@@ -18,8 +18,8 @@ from __future__ import annotations
 
 import importlib
 
-_API = {"MoeLayer", "Router", "Experts", "quantize", "dequantize", "route", "residual_rmsnorm",
-        "device_status", "forward_views"}
+_API = {"MoeLayer", "Router", "Experts", "quantize", "dequantize", "route", "permute", "residual_rmsnorm",
+        "device_status", "forward_views", "unscaled_hidden"}
 _CAPI = {"NVFP4Error", "check", "status_string"}
 
 __all__ = sorted(_API | _CAPI | {"capi", "build"})

@@ -125,6 +125,23 @@ def route(x: torch.Tensor, router: Router, stream=None):
     return ids, w
 
 
+def permute(ids: torch.Tensor, stream=None):
+    """int32 [T, 8] expert ids -> (counts int32 [E], offsets int32 [E+1],
+    sorted_slot int32 [T*8], slot_pos int32 [T*8])."""
+    if ids.dtype != torch.int32 or ids.dim() != 2 or ids.shape[1] != TOP_K:
+        raise ValueError("ids must be an int32 tensor [T, 8]")
+    T = ids.shape[0]
+    dev = ids.device
+    counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    sorted_slot = torch.empty((T * TOP_K,), dtype=torch.int32, device=dev)
+    slot_pos = torch.empty((T * TOP_K,), dtype=torch.int32, device=dev)
+    ws = _workspace(capi.moe_permute_workspace_bytes(T), dev)
+    check(capi.moe_permute(_ptr(ids), T, _ptr(counts), _ptr(offsets), _ptr(sorted_slot), _ptr(slot_pos),
+                           _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+    return counts, offsets, sorted_slot, slot_pos
+
+
 # ------------------------------------------------------------------- forward
 class MoeLayer:
     """One NVFP4 MoE branch: holds the device parameters and a workspace sized
@@ -181,8 +198,17 @@ def forward_views(layer: MoeLayer, T: int) -> dict:
         "offsets": view(v.offsets, E + 1, torch.int32),
         "sorted_slot": view(v.sorted_slot, S, torch.int32),
         "slot_pos": view(v.slot_pos, S, torch.int32),
+        "xexp": view(v.xexp, S, torch.int32),
         "h": view(v.h, S * I, torch.float16).view(S, I),
     }
+
+
+def unscaled_hidden(views: dict) -> torch.Tensor:
+    """The gated hidden h of forward_views in fp32 and at its true scale: row
+    p of the stored h carries the factor 2^(-2 e), e = xexp[p] clamped to
+    [-63, 63]."""
+    e = views["xexp"].clamp(-63, 63).to(torch.float64)
+    return (views["h"].to(torch.float64) * torch.pow(2.0, 2.0 * e)[:, None])
 
 
 def residual_rmsnorm(res: torch.Tensor, y: torch.Tensor | None, x_out: torch.Tensor, eps: float = 1e-6,

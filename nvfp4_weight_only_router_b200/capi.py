@@ -22,6 +22,7 @@ c_void_p, c_int32, c_int64, c_size_t, c_float = (ctypes.c_void_p, ctypes.c_int32
 STATUS = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_ALIGNMENT", 3: "NVFP4_ERR_WORKSPACE",
     4: "NVFP4_ERR_CUDA", 5: "NVFP4_ERR_TIMEOUT", 6: "NVFP4_ERR_UNSUPPORTED", 7: "NVFP4_ERR_DEVICE",
+    8: "NVFP4_ERR_RANGE",
 }
 NVFP4_OK = 0
 NVFP4_ERR_INVALID_ARG = 1
@@ -31,6 +32,7 @@ NVFP4_ERR_CUDA = 4
 NVFP4_ERR_TIMEOUT = 5
 NVFP4_ERR_UNSUPPORTED = 6
 NVFP4_ERR_DEVICE = 7
+NVFP4_ERR_RANGE = 8
 
 
 class moe_router(ctypes.Structure):
@@ -48,7 +50,7 @@ class moe_experts(ctypes.Structure):
 class moe_forward_views(ctypes.Structure):
     _fields_ = [("ids", c_size_t), ("weights", c_size_t), ("counts", c_size_t),
                 ("offsets", c_size_t), ("sorted_slot", c_size_t), ("slot_pos", c_size_t),
-                ("h", c_size_t)]
+                ("xexp", c_size_t), ("h", c_size_t)]
 
 
 _R = ctypes.POINTER(moe_router)
@@ -70,8 +72,13 @@ SIGNATURES = {
     "moe_nvfp4_forward_profiled": (c_int32, [c_void_p, c_int32, _X, _R, c_void_p, c_void_p, c_size_t,
                                              c_void_p, ctypes.POINTER(c_void_p)]),
     "moe_forward_workspace_views": (c_int32, [c_int32, _X, _R, ctypes.POINTER(moe_forward_views)]),
+    "moe_permute_workspace_bytes": (c_size_t, [c_int32]),
+    "moe_permute": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                              c_void_p]),
     "moe_residual_rmsnorm": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_float, c_void_p]),
     "nvfp4_get_device_status": (c_int32, [c_void_p]),
+    "nvfp4_selftest_wait_timeout": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                              c_void_p, c_size_t, ctypes.c_uint32, c_void_p]),
     "nvfp4_status_string": (ctypes.c_char_p, [c_int32]),
     "nvfp4_abi_version": (ctypes.c_int, []),
     "nvfp4_last_cuda_error": (ctypes.c_char_p, []),

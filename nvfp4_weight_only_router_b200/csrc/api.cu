@@ -1,7 +1,6 @@
 // C ABI of the NVFP4 MoE library: argument validation, workspace layout and
 // launch sequencing on the caller's stream.  See include/nvfp4moe.h.
 #include <cmath>
-#include <cstdlib>
 #include <mutex>
 
 #include "../../include/nvfp4moe.h"
@@ -55,60 +54,54 @@ struct Alloc {
   }
 };
 
-struct RouteLayout {
-  int ntiles = 0;
-  bool few_tokens = false;
-  Region counters, logits;
-};
-
-RouteLayout route_layout(Alloc& al, int T) {
-  RouteLayout L;
-  L.ntiles = (T + 15) / 16;
-  L.few_tokens = T <= 256;
-  L.counters = al.take(sizeof(int) * L.ntiles);
-  L.logits = al.take(sizeof(float) * (size_t)T * kE);
-  return L;
-}
-
 constexpr int kFusedPermuteMaxSlots = 1024;  // the router's last CTA groups the slots
 
 // Largest token count that takes the streaming GEMV path; above it the
-// tensor-core grouped GEMMs run.  NVFP4MOE_STREAM_MAX_T overrides the default
-// (read once per process) so the crossover can be re-measured.
-int stream_max_tokens() {
-  static const int v = [] {
-    const char* e = std::getenv("NVFP4MOE_STREAM_MAX_T");
-    return e ? std::atoi(e) : 256;
-  }();
-  return v;
-}
+// tensor-core grouped GEMMs run.
+constexpr int kStreamMaxTokens = 256;
 
 struct FwdLayout {
   Region meta;
-  RouteLayout route;
-  Region ids, wts, chunk_count, sorted, pos, xs, h, obuf;
+  Region ids, wts, chunk_count, sorted, pos, xexp, xs, h, obuf;
   int S = 0, nchunks = 0;
   size_t total = 0;
 };
-
 
 FwdLayout fwd_layout(int T) {
   FwdLayout L;
   Alloc al;
   L.S = T * kTopK;
   L.nchunks = (L.S + 1023) / 1024;
-  // zeroed on entry: meta (includes the permute counter) and the router counters
+  // zeroed on entry: meta (includes the router's arrival counter)
   L.meta = al.take(sizeof(int) * kMetaInts);
-  L.route = route_layout(al, T);
   L.ids = al.take(sizeof(int) * L.S);
   L.wts = al.take(sizeof(float) * L.S);
   L.chunk_count = al.take(sizeof(int) * (size_t)L.nchunks * kE);
   L.sorted = al.take(sizeof(int) * L.S);
   L.pos = al.take(sizeof(int) * L.S);
+  L.xexp = al.take(sizeof(int) * L.S);
   L.xs = al.take(sizeof(__half) * (size_t)L.S * kH);
   L.h = al.take(sizeof(__half) * (size_t)L.S * kI);
   // per-slot outputs, summed in slot order by the combine: deterministic
   L.obuf = al.take(sizeof(float) * (size_t)L.S * kH);
+  L.total = al.cur;
+  return L;
+}
+
+// Permutation workspace of moe_permute: the meta block and the per-chunk counts.
+struct PermLayout {
+  Region meta, chunk_count;
+  int S = 0, nchunks = 0;
+  size_t total = 0;
+};
+
+PermLayout perm_layout(int T) {
+  PermLayout L;
+  Alloc al;
+  L.S = T * kTopK;
+  L.nchunks = (L.S + 1023) / 1024;
+  L.meta = al.take(sizeof(int) * kMetaInts);
+  L.chunk_count = al.take(sizeof(int) * (size_t)L.nchunks * kE);
   L.total = al.cur;
   return L;
 }
@@ -128,12 +121,15 @@ nvfp4_status cuda_fail(cudaError_t e) {
 
 nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : cuda_fail(e); }
 
+// hidden sizes the router kernels take: 8 to 16 slices of 256
+bool router_hidden_ok(int H) { return H % 256 == 0 && H >= 2048 && H <= 4096; }
+
 nvfp4_status check_router(const moe_router* r, bool forward) {
   if (!r || !r->proj || !r->scale || !r->per_expert_scale) return NVFP4_ERR_INVALID_ARG;
   if (r->E <= 0 || r->H <= 0 || r->top_k <= 0 || !(r->eps >= 0.f) || !std::isfinite(r->eps))
     return NVFP4_ERR_INVALID_ARG;
   if (r->E != kE || r->top_k != kTopK) return NVFP4_ERR_UNSUPPORTED;
-  if (forward ? (r->H != kH) : (r->H % kSegK != 0 || r->H > 16384)) return NVFP4_ERR_UNSUPPORTED;
+  if (forward ? (r->H != kH) : !router_hidden_ok(r->H)) return NVFP4_ERR_UNSUPPORTED;
   if (!aligned(r->proj, 16) || !aligned(r->scale, 16) || !aligned(r->per_expert_scale, 16) ||
       (r->logit_bias && !aligned(r->logit_bias, 16)))
     return NVFP4_ERR_ALIGNMENT;
@@ -152,8 +148,7 @@ nvfp4_status check_experts(const moe_experts* x) {
   return NVFP4_OK;
 }
 
-RouteArgs make_route_args(const void* x, int T, const moe_router* r, const RouteLayout& L, void* ws,
-                          int32_t* ids, float* wts, int* status) {
+RouteArgs make_route_args(const void* x, int T, const moe_router* r, int32_t* ids, float* wts, int* status) {
   RouteArgs a;
   a.x = static_cast<const uint16_t*>(x);
   a.proj = static_cast<const uint16_t*>(r->proj);
@@ -162,11 +157,9 @@ RouteArgs make_route_args(const void* x, int T, const moe_router* r, const Route
   a.bias = r->logit_bias;
   a.T = T;
   a.H = r->H;
-  a.few_tokens = L.few_tokens;
+  a.few_tokens = T <= 256;
   a.eps = r->eps;
   a.inv_sqrt_h = (float)(1.0 / std::sqrt((double)r->H));
-  a.logits = at<float>(ws, L.logits);
-  a.tile_counter = at<int>(ws, L.counters);
   a.ids = ids;
   a.wts = wts;
   a.meta = nullptr;
@@ -177,6 +170,8 @@ RouteArgs make_route_args(const void* x, int T, const moe_router* r, const Route
 }
 
 }  // namespace
+
+int nvfp4moe::fail_cuda(cudaError_t e) { return cuda_fail(e); }
 
 extern "C" {
 
@@ -194,6 +189,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_TIMEOUT: return "device wait timed out";
     case NVFP4_ERR_UNSUPPORTED: return "unsupported shape";
     case NVFP4_ERR_DEVICE: return "invalid data detected on the device";
+    case NVFP4_ERR_RANGE: return "an activation left the range of the f16 tensor-core operands";
   }
   return "unknown status";
 }
@@ -239,9 +235,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* q, const uint8_t* s, const float* g
 // ------------------------------------------------------------------- route
 size_t moe_route_workspace_bytes(int32_t T, const moe_router* r) {
   if (T < 1 || T > 65536 || check_router(r, false) != NVFP4_OK) return 0;
-  Alloc al;
-  route_layout(al, T);
-  return al.cur;
+  return 256;  // the router kernels keep their scratch on chip
 }
 
 nvfp4_status moe_route(const void* x, int32_t T, const moe_router* r, int32_t* ids, float* w,
@@ -250,16 +244,43 @@ nvfp4_status moe_route(const void* x, int32_t T, const moe_router* r, int32_t* i
   nvfp4_status st = check_router(r, false);
   if (st != NVFP4_OK) return st;
   if (!aligned(x, 16) || !aligned(ids, 16) || !aligned(w, 16)) return NVFP4_ERR_ALIGNMENT;
-  const size_t need = moe_route_workspace_bytes(T, r);
-  if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
+  if (!ws || ws_bytes < moe_route_workspace_bytes(T, r)) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
-  Alloc al;
-  RouteLayout L = route_layout(al, T);
+  RouteArgs a = make_route_args(x, T, r, ids, w, device_status_ptr());
+  return cuda_status(launch_route(a, as_stream(stream)));
+}
+
+// ---------------------------------------------------------------- permute
+size_t moe_permute_workspace_bytes(int32_t T) {
+  if (T < 1 || T > 65536) return 0;
+  return perm_layout(T).total;
+}
+
+nvfp4_status moe_permute(const int32_t* ids, int32_t T, int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
+                         int32_t* slot_pos, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 1 || T > 65536 || !ids || !counts || !offsets || !sorted_slot || !slot_pos) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(ids, 16) || !aligned(counts, 16) || !aligned(offsets, 16) || !aligned(sorted_slot, 16) ||
+      !aligned(slot_pos, 16))
+    return NVFP4_ERR_ALIGNMENT;
+  const PermLayout L = perm_layout(T);
+  if (!ws || ws_bytes < L.total) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
   cudaStream_t s = as_stream(stream);
-  cudaError_t e = cudaMemsetAsync(at<int>(ws, L.counters), 0, L.counters.bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  RouteArgs a = make_route_args(x, T, r, L, ws, ids, w, device_status_ptr());
-  return cuda_status(launch_route(a, s));
+  PermuteArgs pa;
+  pa.ids = ids;
+  pa.S = L.S;
+  pa.nchunks = L.nchunks;
+  pa.meta = at<int>(ws, L.meta);
+  pa.chunk_count = at<int>(ws, L.chunk_count);
+  pa.sorted_slot = sorted_slot;
+  pa.slot_pos = slot_pos;
+  pa.status = device_status_ptr();
+  cudaError_t e = launch_permute(pa, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(counts, pa.meta + kMetaCounts, sizeof(int) * kE, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(offsets, pa.meta + kMetaOffsets, sizeof(int) * (kE + 1), cudaMemcpyDeviceToDevice, s);
+  return cuda_status(e);
 }
 
 // ----------------------------------------------------------------- forward
@@ -282,6 +303,7 @@ nvfp4_status moe_forward_workspace_views(int32_t T, const moe_experts* ex, const
   out->offsets = L.meta.off + sizeof(int) * kMetaOffsets;
   out->sorted_slot = L.sorted.off;
   out->slot_pos = L.pos.off;
+  out->xexp = L.xexp.off;
   out->h = L.h.off;
   return NVFP4_OK;
 }
@@ -312,15 +334,13 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   };
   if (!mark(0)) return cuda_fail(cudaGetLastError());
 
-  // meta and router counters are contiguous at the start of the workspace
-  const size_t zero_bytes = L.route.counters.off + L.route.counters.bytes;
-  cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, s);
+  cudaError_t e = cudaMemsetAsync(at<int>(ws, L.meta), 0, L.meta.bytes, s);
   if (e != cudaSuccess) return cuda_fail(e);
 
   int32_t* ids = at<int32_t>(ws, L.ids);
   float* wts = at<float>(ws, L.wts);
-  RouteArgs ra = make_route_args(x, T, r, L.route, ws, ids, wts, status);
-  const bool fused_permute = L.S <= kFusedPermuteMaxSlots;
+  RouteArgs ra = make_route_args(x, T, r, ids, wts, status);
+  const bool fused_permute = ra.few_tokens && L.S <= kFusedPermuteMaxSlots;
   if (fused_permute) {
     ra.meta = at<int>(ws, L.meta);
     ra.sorted_slot = at<int>(ws, L.sorted);
@@ -351,6 +371,7 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   xa.sorted_slot = pa.sorted_slot;
   xa.slot_pos = pa.slot_pos;
   xa.wts = wts;
+  xa.xexp = at<int>(ws, L.xexp);
   xa.h = at<__half>(ws, L.h);
   xa.obuf = at<float>(ws, L.obuf);
   xa.y = y;
@@ -361,7 +382,7 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   // the activations follow their slots into expert order (f16 for the MMAs)
   if ((e = launch_gather_sorted(xa, s)) != cudaSuccess) return cuda_fail(e);
   if (!mark(2)) return cuda_fail(cudaGetLastError());
-  if (T <= stream_max_tokens()) {
+  if (T <= kStreamMaxTokens) {
     // few tokens per expert: the weight stream bounds the step (streaming
     // GEMV with register dequantisation)
     e = launch_gate_up_stream(xa, s);
@@ -389,6 +410,21 @@ nvfp4_status moe_nvfp4_forward_profiled(const void* x, int32_t T, const moe_expe
                                         const moe_router* r, void* y, void* ws, size_t ws_bytes,
                                         void* stream, void* const* phase_events) {
   return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, phase_events);
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(const void* w, int64_t E, int64_t N, int64_t K, uint8_t* q, uint8_t* s,
+                                         float* g, void* ws, size_t ws_bytes, uint32_t limit_us, void* stream) {
+  nvfp4_status st = check_quant_dims(E, N, K);
+  if (st != NVFP4_OK) return st;
+  if (!w || !q || !s || !g || limit_us < 1 || limit_us > 1000000) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(q, 16) || !aligned(s, 16) || !aligned(g, 16)) return NVFP4_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < nvfp4_quantize_workspace_bytes(E, N, K)) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
+  const cudaError_t e = launch_quantize_timeout_selftest(
+      static_cast<const uint16_t*>(w), E, N, K, q, s, g, static_cast<uint32_t*>(ws),
+      (int64_t)(ws_bytes / sizeof(uint32_t)), device_status_ptr(), (uint64_t)limit_us * 1000ull, as_stream(stream));
+  if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
+  return cuda_status(e);
 }
 
 // ------------------------------------------------------------ chain helper

@@ -31,6 +31,7 @@ constexpr int kDnSegs = (kI + kSegK - 1) / kSegK; // 6 (the last one half full)
 // Device status codes (mirror nvfp4_status).
 constexpr int kStatusTimeout = 5;
 constexpr int kStatusDevice = 7;
+constexpr int kStatusRange = 8;
 
 // Layout of the small integer "meta" block at the start of a forward
 // workspace.
@@ -78,11 +79,28 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 __device__ __forceinline__ uint32_t bcast_lo(uint32_t v) { return __byte_perm(v, v, 0x1010); }
 __device__ __forceinline__ uint32_t bcast_hi(uint32_t v) { return __byte_perm(v, v, 0x3232); }
 
-// fp32 -> f16 with saturation to +-65504 (finite inputs).
-__device__ __forceinline__ __half f32_to_f16_sat(float v) {
+// fp32 -> f16 with saturation to +-65504 (finite inputs); `over` is set
+// when the value lies beyond the f16 range (|v| >= 65520 would round to
+// infinity), i.e. when the saturation changed the result.
+__device__ __forceinline__ __half f32_to_f16_sat(float v, bool& over) {
+  over |= fabsf(v) >= 65520.0f;
   v = fminf(fmaxf(v, -65504.0f), 65504.0f);
   return __float2half_rn(v);
 }
+
+// 2^k as an fp32 value, for -126 <= k <= 127 (exact).
+__device__ __forceinline__ float exp2i(int k) { return __int_as_float((k + 127) << 23); }
+
+// Power-of-two prescale of the expert GEMMs' f16 operands.  Token t's
+// activation row enters the tensor cores as x * 2^(15 - e_t) and its gated
+// hidden rows as h * 2^(-2 e_h), with e_t = floor(log2 max|x_t|) clamped to
+// [kXExpMin, kXExpMax] and e_h = e_t clamped to [-kHExpLim, kHExpLim]; the
+// epilogues multiply the fp32 accumulators back by the inverse powers of two,
+// so the scaling is exact.  Scaled, every bf16 element of a row whose maximum
+// lies in [2^-111, 2^113) is exact in f16 down to 2^-32 of the row maximum,
+// and h keeps its f16 precision whatever the magnitude of x (h grows as x^2).
+constexpr int kXExpMin = -111, kXExpMax = 112, kHExpLim = 63;
+__device__ __forceinline__ int h_exp(int e) { return max(-kHExpLim, min(kHExpLim, e)); }
 
 __device__ __forceinline__ uint32_t pack_f16x2(__half lo, __half hi) {
   return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
@@ -226,17 +244,6 @@ __device__ __forceinline__ uint4 lds_v4(const void* p) {
       : "r"(smem_u32(p))
       : "memory");
   return v;
-}
-
-__device__ __forceinline__ uint16_t lds_u16(const void* p) {
-  uint16_t v;
-  asm("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-
-// named barrier among `nthreads` threads (multiple of 32)
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace nvfp4moe

@@ -13,8 +13,24 @@ namespace nvfp4moe {
 cudaError_t launch_quantize(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* q,
                             uint8_t* s, float* g, uint32_t* amax_ws, int64_t ws_words, int* status,
                             cudaStream_t st);
+// The single-pass kernel of launch_quantize with a cross-CTA arrival count
+// that cannot be met and every wait limited to wait_ns: the failure path of
+// the bounded waits (cudaErrorNotSupported if the shape does not take the
+// single-pass kernel).
+cudaError_t launch_quantize_timeout_selftest(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* q,
+                                             uint8_t* s, float* g, uint32_t* amax_ws, int64_t ws_words,
+                                             int* status, uint64_t wait_ns, cudaStream_t st);
 // the library's device status word of the current device (null on failure)
 int* device_status_ptr();
+// Record `e` as the calling thread's last CUDA error (what
+// nvfp4_last_cuda_error reports) and return NVFP4_ERR_CUDA.
+int fail_cuda(cudaError_t e);
+// Raise a kernel's dynamic shared-memory limit to smem_bytes (and allow
+// non-portable cluster sizes if asked) once per kernel and device; safe to
+// call from several host threads.
+cudaError_t configure_kernel_once(const void* fn, int smem_bytes, bool nonportable_cluster = false);
+// Number of SMs of the current device.
+cudaError_t sm_count(int* sms);
 cudaError_t launch_dequantize(const uint8_t* q, const uint8_t* s, const float* g, int64_t E,
                               int64_t N, int64_t K, float* out, cudaStream_t st);
 
@@ -24,15 +40,13 @@ struct RouteArgs {
   const uint16_t* scale;  // bf16 [H]
   const uint16_t* pes;    // bf16 [E]
   const float* bias;      // f32 [E] or null
-  int T, H;
-  bool few_tokens;        // 16 CTAs of 8 experts per token tile (else 1 CTA of 128)
+  int T, H;               // H: 8 to 16 slices of 256
+  bool few_tokens;        // T <= 256: clusters of H/256 CTAs per 16 tokens (else 32 tokens per CTA)
   float eps, inv_sqrt_h;
-  float* logits;          // [T, 128] scratch
-  int* tile_counter;      // [ceil(T/16)], zero on entry, left zero
   int32_t* ids;           // [T, 8]
   float* wts;             // [T, 8]
-  // optional fused permutation (T*8 <= 1024): meta (route counter zero on
-  // entry), sorted_slot [T*8], slot_pos [T*8]; meta == null -> not fused
+  // optional fused permutation (few tokens, T*8 <= 1024): meta (route counter
+  // zero on entry), sorted_slot [T*8], slot_pos [T*8]; meta == null -> not fused
   int* meta;
   int* sorted_slot;
   int* slot_pos;
@@ -61,6 +75,9 @@ struct ExpertArgs {
   const uint16_t* x;        // bf16 [T, H] (the layer input)
   __half* xs;               // [S, H] activations in expert-sorted slot order
   const int* meta;
+  // [S] per sorted slot: e_t of the slot's token (the f16 operand prescale:
+  // x enters as x * 2^(15 - e_t), h as h * 2^(-2 h_exp(e_t)))
+  int* xexp;
   const int* sorted_slot;   // [S]
   const int* slot_pos;      // [S]
   const float* wts;         // [S]

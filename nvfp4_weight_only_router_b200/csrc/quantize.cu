@@ -33,30 +33,33 @@ namespace nvfp4moe {
 // |w| of a bf16 pattern as a monotone integer key (non-NaN inputs).
 __device__ __forceinline__ uint32_t bf16_abs_key(uint32_t b) { return b & 0x7FFFu; }
 
-__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ w, int64_t per_expert,
+// Per-tensor max |w|, tensors on grid rows blockIdx.y, blockIdx.y + gridDim.y, ...
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ w, int64_t E, int64_t per_expert,
                                                    uint32_t* __restrict__ amax_bits) {
-  const int e = blockIdx.y;
-  const uint4* base = reinterpret_cast<const uint4*>(w + (size_t)e * per_expert);
-  const int64_t n16 = per_expert / 8;  // 8 bf16 per 16-byte load
-  uint32_t m = 0;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    uint4 v = ldg_nc_v4(base + i);
-    uint32_t a[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      m = max(m, bf16_abs_key(a[j] & 0xFFFFu));
-      m = max(m, bf16_abs_key(a[j] >> 16));
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
   __shared__ uint32_t red[8];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int j = 1; j < (int)(blockDim.x >> 5); ++j) m = max(m, red[j]);
-    atomicMax(amax_bits + e, m << 16);  // fp32 bit pattern of the bf16 amax
+  const int64_t n16 = per_expert / 8;  // 8 bf16 per 16-byte load
+  for (int64_t e = blockIdx.y; e < E; e += gridDim.y) {
+    const uint4* base = reinterpret_cast<const uint4*>(w + (size_t)e * per_expert);
+    uint32_t m = 0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+         i += (int64_t)gridDim.x * blockDim.x) {
+      uint4 v = ldg_nc_v4(base + i);
+      uint32_t a[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m = max(m, bf16_abs_key(a[j] & 0xFFFFu));
+        m = max(m, bf16_abs_key(a[j] >> 16));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int j = 1; j < (int)(blockDim.x >> 5); ++j) m = max(m, red[j]);
+      atomicMax(amax_bits + e, m << 16);  // fp32 bit pattern of the bf16 amax
+    }
+    __syncthreads();  // red[] is reused by the next tensor
   }
 }
 
@@ -255,9 +258,15 @@ __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
 //   compute: full(e+2) -> reduce -> part(e+2) -> scale(e) -> encode e -> free(e)
 // A CTA publishes e+1 only after all CTAs published e-1, so counters modulo 3
 // never mix tensors that are both in flight.
+//
+// extra_target (0 in normal use) raises the arrival count the control thread
+// waits for, and wait_ns limits every wait: with extra_target > 0 the wait
+// can never be met, which exercises the timeout path (every CTA gives up,
+// records the timeout status, lets its copies land and exits).
 __global__ void __launch_bounds__(kQThreads, 1)
     quantize_fused_kernel(const uint16_t* __restrict__ w, int E, int64_t bpe, uint32_t* amax_ws,
-                          uint8_t* __restrict__ q, uint8_t* __restrict__ s, float* __restrict__ g, int* status) {
+                          uint8_t* __restrict__ q, uint8_t* __restrict__ s, float* __restrict__ g, int* status,
+                          uint32_t extra_target, uint64_t wait_ns) {
   extern __shared__ __align__(128) uint8_t qsm[];
   uint64_t* full = reinterpret_cast<uint64_t*>(qsm);        // copy landed
   uint64_t* part = full + kQBufs;                           // compute warps' maxima written
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       // publish tensor t's maximum once the compute warps have reduced it
       auto contribute = [&](int t) -> bool {
         const int b = t % kQBufs;
-        if (*abort_flag || !mbar_wait_bounded(&part[b], (t / kQBufs) & 1)) return false;
+        if (*abort_flag || !mbar_wait_bounded(&part[b], (t / kQBufs) & 1, wait_ns)) return false;
         uint32_t m = 0;
         for (int j = 0; j < kQCompute / 32; ++j) m = max(m, red[b][j]);
         atomicMax(amax_ws + t, m << 16);  // fp32 bit pattern of the bf16 amax
@@ -317,7 +326,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (!contribute(0)) fail();
       for (int e = 0; e < E && !*abort_flag; ++e) {
         const int b = e % kQBufs;
-        const uint32_t target = (uint32_t)n * (uint32_t)(e / 3 + 1);
+        const uint32_t target = (uint32_t)n * (uint32_t)(e / 3 + 1) + extra_target;
         uint32_t c = ld_acquire_u32(ctr + e % 3);  // in flight while tensor e+1 is published
         if (e + 1 < E && !contribute(e + 1)) {
           fail();
@@ -326,7 +335,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (c < target) {
           const uint64_t t0 = globaltimer_ns();
           while ((c = ld_acquire_u32(ctr + e % 3)) < target)
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+            if (globaltimer_ns() - t0 > wait_ns) break;
         }
         if (c < target) {
           fail();
@@ -337,7 +346,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         mbar_arrive(&scl[b]);
         const int t = e + kQBufs - 1;
         if (t < E) {
-          if (t >= kQBufs && !mbar_wait_bounded(&freeb[t % kQBufs], ((t - kQBufs) / kQBufs) & 1)) {
+          if (t >= kQBufs && !mbar_wait_bounded(&freeb[t % kQBufs], ((t - kQBufs) / kQBufs) & 1, wait_ns)) {
             fail();
             break;
           }
@@ -355,7 +364,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int ct = tid - 32, cw = warp - 1;
     auto reduce = [&](int t) -> bool {  // |w| over tensor t's piece -> red[t % 4][cw]
       const int b = t % kQBufs;
-      if (!mbar_wait_bounded(&full[b], (t / kQBufs) & 1)) return false;
+      if (!mbar_wait_bounded(&full[b], (t / kQBufs) & 1, wait_ns)) return false;
       const uint4* v = reinterpret_cast<const uint4*>(buf0 + (size_t)b * kQMaxPiece);
       uint32_t m = 0;
       for (int i = ct; i < nb * 2; i += kQCompute) {
@@ -379,7 +388,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         break;
       }
       const int b = e % kQBufs;
-      if (!mbar_wait_bounded(&scl[b], (e / kQBufs) & 1)) {
+      if (!mbar_wait_bounded(&scl[b], (e / kQBufs) & 1, wait_ns)) {
         ok = false;
         break;
       }
@@ -432,42 +441,52 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
   dst[1] = o1;
 }
 
+namespace {
+
+constexpr int kQSmem = kQHeader + kQBufs * kQMaxPiece;
+static_assert(kQSmem <= 232448, "shared memory budget of the single-pass quantiser");
+
+// the single-pass kernel applies: the largest piece fits a buffer, every CTA
+// gets a few blocks, and the workspace holds the arrival counters
+bool single_pass_fits(int64_t E, int64_t bpe, int64_t ws_words, int sms) {
+  return ws_words >= E + 3 && E <= (int64_t(1) << 24) && bpe >= 8 * (int64_t)sms &&
+         (bpe + sms - 1) / sms * 32 <= kQMaxPiece;
+}
+
+cudaError_t launch_fused(const uint16_t* w, int64_t E, int64_t bpe, uint32_t* amax_ws, uint8_t* q, uint8_t* s,
+                         float* g, int* status, int sms, uint32_t extra_target, uint64_t wait_ns,
+                         cudaStream_t st) {
+  cudaError_t err = configure_kernel_once((const void*)quantize_fused_kernel, kQSmem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)sms);
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = (size_t)kQSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the arrival waits end
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_fused_kernel, w, (int)E, bpe, amax_ws, q, s, g, status, extra_target,
+                            wait_ns);
+}
+
+}  // namespace
+
 cudaError_t launch_quantize(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* q,
                             uint8_t* s, float* g, uint32_t* amax_ws, int64_t ws_words, int* status,
                             cudaStream_t st) {
   const int64_t per = N * K;
   const int64_t bpe = per / 16;
-  int dev = 0, sms = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  int sms = 0;
+  cudaError_t err = sm_count(&sms);
   if (err != cudaSuccess) return err;
-  err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (err != cudaSuccess) return err;
-  // single pass: the largest piece must fit a buffer, every CTA should get a
-  // few blocks, and the workspace must hold the arrival counters
-  const bool fused = ws_words >= E + 3 && E <= (int64_t(1) << 24) && bpe >= 8 * (int64_t)sms &&
-                     (bpe + sms - 1) / sms * 32 <= kQMaxPiece;
-  static_assert(kQHeader + kQBufs * kQMaxPiece <= 232448, "shared memory budget of the single-pass quantiser");
+  const bool fused = single_pass_fits(E, bpe, ws_words, sms);
   err = cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * (size_t)(fused ? E + 3 : E), st);
   if (err != cudaSuccess) return err;
   if (fused) {
-    static int configured_dev = -1;
-    const int smem = kQHeader + kQBufs * kQMaxPiece;
-    if (configured_dev != dev) {
-      err = cudaFuncSetAttribute(quantize_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (err != cudaSuccess) return err;
-      configured_dev = dev;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)sms);
-    cfg.blockDim = dim3(kQThreads);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the arrival waits end
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, quantize_fused_kernel, w, (int)E, bpe, amax_ws, q, s, g, status);
+    err = launch_fused(w, E, bpe, amax_ws, q, s, g, status, sms, 0u, kWaitTimeoutNs, st);
     // not every SM available to this context (a partitioned GPU): the two
     // passes below need no co-residency (their amax words are cleared too)
     if (err != cudaErrorCooperativeLaunchTooLarge) return err;
@@ -475,12 +494,26 @@ cudaError_t launch_quantize(const uint16_t* w, int64_t E, int64_t N, int64_t K, 
   }
   int gx = (int)((per / 8 + 255) / 256);
   if (gx > 64) gx = 64;
-  amax_kernel<<<dim3(gx, (unsigned)E), 256, 0, st>>>(w, per, amax_ws);
+  const unsigned gy = (unsigned)(E < 65535 ? E : 65535);  // tensors beyond: grid-stride
+  amax_kernel<<<dim3(gx, gy), 256, 0, st>>>(w, E, per, amax_ws);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int64_t nb = E * bpe;
   encode_kernel<<<(unsigned)((nb + 255) / 256), 256, 0, st>>>(w, bpe, nb, amax_ws, q, s, g);
   return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_timeout_selftest(const uint16_t* w, int64_t E, int64_t N, int64_t K, uint8_t* q,
+                                             uint8_t* s, float* g, uint32_t* amax_ws, int64_t ws_words,
+                                             int* status, uint64_t wait_ns, cudaStream_t st) {
+  const int64_t bpe = N * K / 16;
+  int sms = 0;
+  cudaError_t err = sm_count(&sms);
+  if (err != cudaSuccess) return err;
+  if (!single_pass_fits(E, bpe, ws_words, sms)) return cudaErrorNotSupported;
+  err = cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * (size_t)(E + 3), st);
+  if (err != cudaSuccess) return err;
+  return launch_fused(w, E, bpe, amax_ws, q, s, g, status, sms, 1u, wait_ns, st);
 }
 
 cudaError_t launch_dequantize(const uint8_t* q, const uint8_t* s, const float* g, int64_t E,

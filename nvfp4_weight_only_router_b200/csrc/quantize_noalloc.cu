@@ -13,7 +13,10 @@
 // plus three arrival counters when the tensors take the single-pass kernel)
 // before it reads them.  Calls
 // that overlap on the GPU race on the array.  Every GPU that loads the
-// library holds the array (16 KiB) until the process exits.
+// library holds the array (16 KiB) until the process exits; with CUDA's lazy
+// module loading the driver places it (with the module's code) at the first
+// call on each device, so callers with a strict no-allocation window make one
+// call before it opens.
 #include <mutex>
 
 #include "../../include/nvfp4moe.h"
@@ -34,17 +37,21 @@ uint32_t* g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
 // Set-up, once per device, with that device current: the device address of
-// the scratch array.  Returns null if the runtime call fails.
-uint32_t* noalloc_scratch() {
+// the scratch array, or the error of the runtime call that failed.
+cudaError_t noalloc_scratch(uint32_t** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (!g_noalloc_ptr[dev]) {
     uint32_t* ptr = nullptr;
-    if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_amax) != cudaSuccess) return nullptr;
+    e = cudaGetSymbolAddress((void**)&ptr, g_noalloc_amax);
+    if (e != cudaSuccess) return e;
     g_noalloc_ptr[dev] = ptr;
   }
-  return g_noalloc_ptr[dev];
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -58,11 +65,12 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* w, int64_t E, int64_t
   if (E > kNoAllocMaxTensors) return NVFP4_ERR_UNSUPPORTED;  // beyond the fixed scratch
   if (!w || !q || !s || !g) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(w) || !aligned16(q) || !aligned16(s) || !aligned16(g)) return NVFP4_ERR_ALIGNMENT;
-  uint32_t* scratch = noalloc_scratch();
-  if (!scratch) return NVFP4_ERR_CUDA;
+  uint32_t* scratch = nullptr;
+  const cudaError_t se = noalloc_scratch(&scratch);
+  if (se != cudaSuccess) return static_cast<nvfp4_status>(nvfp4moe::fail_cuda(se));
   // launch_quantize clears the scratch words it uses before the amax pass
   const cudaError_t e = nvfp4moe::launch_quantize(static_cast<const uint16_t*>(w), E, N, K, q, s, g,
                                                   scratch, kNoAllocMaxTensors, nvfp4moe::device_status_ptr(),
                                                   static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+  return e == cudaSuccess ? NVFP4_OK : static_cast<nvfp4_status>(nvfp4moe::fail_cuda(e));
 }

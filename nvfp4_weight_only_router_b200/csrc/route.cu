@@ -10,20 +10,17 @@
 // bf16 MMAs (hi and lo against the same proj fragment) accumulate the exact
 // products in fp32.
 //
-// Work split: a CTA (8 warps) owns 16 tokens x EG experts.
-//   EG = 8 (few tokens): 16 CTAs per token tile, the 8 warps split K and meet
-//        in shared memory, so each CTA reads only 8 rows of proj and the 720 KB
-//        of proj are spread over 16 SMs per tile;
-//   EG = 128 (many tokens): one CTA per token tile, warp w owns experts
-//        [16w, 16w+16) over all of K.
-// The complete logits go to the workspace; the last CTA of a token tile
-// (arrival counter) runs softmax / top-8 for its 16 tokens, one warp per two
-// tokens.  With few tokens (T*8 <= 1024) the last tile to finish also groups
-// the slots by expert (the permutation step) in the same launch.
+// Two kernels:
+//   few tokens (T <= 256): a thread-block cluster per 16 tokens, one CTA per
+//        256-wide K slice, partial logits summed through distributed shared
+//        memory in rank order; the last CTA of the launch also groups the
+//        slots by expert (the permutation step) when T*8 <= 1024;
+//   many tokens: one CTA per 32 tokens over the whole K, streamed through a
+//        TMA ring.
+// Both run softmax / top-8 with one warp per token and write ids and weights.
 //
-// Within a 128-element K segment, lane quad q holds elements [32q, 32q+32);
-// MMA step j takes elements 32q+4j+{0,1} as the fragment's low k-pair and
-// 32q+4j+{2,3} as its high k-pair, for both operands.
+// Within a K block, the MMA fragments follow the warp-level m16n8k16 layout
+// (ldmatrix from 128B-swizzled shared-memory tiles).
 #include "tc_common.cuh"
 #include "kernels.h"
 
@@ -32,14 +29,6 @@ namespace nvfp4moe {
 namespace {
 
 constexpr int kRouteThreads = 256;
-
-__device__ __forceinline__ void split_hi_lo(float p0, float p1, uint32_t& hi, uint32_t& lo) {
-  const __nv_bfloat16 h0 = __float2bfloat16_rn(p0), h1 = __float2bfloat16_rn(p1);
-  const __nv_bfloat16 l0 = __float2bfloat16_rn(p0 - __bfloat162float(h0));
-  const __nv_bfloat16 l1 = __float2bfloat16_rn(p1 - __bfloat162float(h1));
-  hi = pack_bf16x2(h0, h1);
-  lo = pack_bf16x2(l0, l1);
-}
 
 // Top-8 of 128 logits held 4 per lane (expert lane + 32 i).  Ordered by
 // descending logit (= descending probability); equal logits -> lower id first.
@@ -214,320 +203,6 @@ __device__ void block_permute_small(const RouteArgs& a) {
     }
     __syncthreads();
   }
-}
-
-template <int EG>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
-  constexpr int KW = EG == 8 ? 8 : 1;   // K-split ways inside the CTA
-  constexpr int NTW = EG == 8 ? 1 : 2;  // 8-expert n-tiles per warp
-  __shared__ float4 s_red[kRouteThreads / 32][NTW][32];
-  __shared__ float s_ss[KW][16];
-  __shared__ int s_last;
-
-  const int tile = blockIdx.x, eg = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-  const int kpart = warp % KW, ngroup = warp / KW;
-  const int e_base = eg * EG + ngroup * NTW * 8;  // first expert of this warp
-  const int t0 = tile * 16 + g, t1 = t0 + 8;
-  const bool v0 = t0 < a.T, v1 = t1 < a.T;
-  const int nseg = a.H / kSegK;
-  const uint16_t* x0 = a.x + (size_t)(v0 ? t0 : 0) * a.H + 32 * q;
-  const uint16_t* x1 = a.x + (size_t)(v1 ? t1 : 0) * a.H + 32 * q;
-  const uint16_t* prow = a.proj + (size_t)(e_base + g) * a.H + 32 * q;
-  const bool do_ss = ngroup == 0;
-
-  float acc[NTW][4];
-#pragma unroll
-  for (int n = 0; n < NTW; ++n)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-  float ss0 = 0.f, ss1 = 0.f;
-
-  for (int seg = kpart; seg < nseg; seg += KW) {
-#pragma unroll
-    for (int sub = 0; sub < 4; ++sub) {
-      const int k = seg * kSegK + 8 * sub;
-      const uint4 zero = make_uint4(0, 0, 0, 0);
-      const uint4 xa = v0 ? ldg_nc_v4(x0 + k) : zero;
-      const uint4 xb = v1 ? ldg_nc_v4(x1 + k) : zero;
-      const uint4 sc = ldg_nc_v4(a.scale + k + 32 * q);
-      uint4 bw[NTW];
-#pragma unroll
-      for (int n = 0; n < NTW; ++n) bw[n] = ldg_nc_v4(prow + (size_t)n * 8 * a.H + k);
-      const uint32_t xaw[4] = {xa.x, xa.y, xa.z, xa.w}, xbw[4] = {xb.x, xb.y, xb.z, xb.w};
-      const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
-      uint32_t hi_a[4], lo_a[4], hi_b[4], lo_b[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float s0 = bf16_bits_to_f32(scw[w] & 0xFFFFu), s1 = bf16_bits_to_f32(scw[w] >> 16);
-        const float xa0 = bf16_bits_to_f32(xaw[w] & 0xFFFFu), xa1 = bf16_bits_to_f32(xaw[w] >> 16);
-        const float xb0 = bf16_bits_to_f32(xbw[w] & 0xFFFFu), xb1 = bf16_bits_to_f32(xbw[w] >> 16);
-        split_hi_lo(__fmul_rn(xa0, s0), __fmul_rn(xa1, s1), hi_a[w], lo_a[w]);
-        split_hi_lo(__fmul_rn(xb0, s0), __fmul_rn(xb1, s1), hi_b[w], lo_b[w]);
-        if (do_ss) {
-          ss0 = __fmaf_rn(xa0, xa0, ss0);
-          ss0 = __fmaf_rn(xa1, xa1, ss0);
-          ss1 = __fmaf_rn(xb0, xb0, ss1);
-          ss1 = __fmaf_rn(xb1, xb1, ss1);
-        }
-      }
-      const uint32_t Ah0[4] = {hi_a[0], hi_b[0], hi_a[1], hi_b[1]};
-      const uint32_t Al0[4] = {lo_a[0], lo_b[0], lo_a[1], lo_b[1]};
-      const uint32_t Ah1[4] = {hi_a[2], hi_b[2], hi_a[3], hi_b[3]};
-      const uint32_t Al1[4] = {lo_a[2], lo_b[2], lo_a[3], lo_b[3]};
-#pragma unroll
-      for (int n = 0; n < NTW; ++n) {
-        mma_bf16_16816(acc[n], Ah0, bw[n].x, bw[n].y);
-        mma_bf16_16816(acc[n], Al0, bw[n].x, bw[n].y);
-        mma_bf16_16816(acc[n], Ah1, bw[n].z, bw[n].w);
-        mma_bf16_16816(acc[n], Al1, bw[n].z, bw[n].w);
-      }
-    }
-  }
-
-  // sum of squares of each token over this warp's K part
-  if (do_ss) {
-    ss0 += __shfl_xor_sync(0xffffffffu, ss0, 1);
-    ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
-    ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
-    ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
-    if (q == 0) {
-      s_ss[kpart][g] = ss0;
-      s_ss[kpart][g + 8] = ss1;
-    }
-  }
-#pragma unroll
-  for (int n = 0; n < NTW; ++n) s_red[warp][n][lane] = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
-  __syncthreads();
-
-  // complete logits of this CTA: warps of K part 0 add the other parts
-  if (kpart == 0) {
-    float ssa = 0.f, ssb = 0.f;
-    for (int p = 0; p < KW; ++p) {
-      ssa += s_ss[p][g];
-      ssb += s_ss[p][g + 8];
-    }
-    const float fa = (1.0f / sqrtf(ssa / (float)a.H + a.eps)) * a.inv_sqrt_h;
-    const float fb = (1.0f / sqrtf(ssb / (float)a.H + a.eps)) * a.inv_sqrt_h;
-#pragma unroll
-    for (int n = 0; n < NTW; ++n) {
-      float4 v = s_red[warp][n][lane];
-      for (int p = 1; p < KW; ++p) {
-        const float4 o = s_red[warp + p][n][lane];
-        v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
-      }
-      const int e = e_base + n * 8 + 2 * q;
-      const float b0 = a.bias ? a.bias[e] : 0.f, b1 = a.bias ? a.bias[e + 1] : 0.f;
-      if (v0)
-        *reinterpret_cast<float2*>(a.logits + (size_t)t0 * kE + e) = make_float2(v.x * fa + b0, v.y * fa + b1);
-      if (v1)
-        *reinterpret_cast<float2*>(a.logits + (size_t)t1 * kE + e) = make_float2(v.z * fb + b0, v.w * fb + b1);
-    }
-  }
-
-  constexpr int kCtasPerTile = kE / EG;
-  if (kCtasPerTile > 1) {
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const int prev = atomicAdd(a.tile_counter + tile, 1);
-      s_last = (prev == kCtasPerTile - 1);
-      if (s_last) a.tile_counter[tile] = 0;  // leave the counter zero for the next call
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-  } else {
-    __syncthreads();
-  }
-
-  // softmax / top-8: warp w handles tokens 2w, 2w+1 of the tile
-  float pesv[4], bv_unused[4];
-  load_expert_consts(a, pesv, bv_unused);
-  for (int j = 0; j < 2; ++j) {
-    const int t = tile * 16 + warp * 2 + j;
-    if (t >= a.T) break;
-    float lg[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) lg[i] = __ldcg(a.logits + (size_t)t * kE + lane + 32 * i);
-    finish_token(a, t, lg, pesv);
-  }
-
-  if (a.meta == nullptr) return;
-  // few tokens: the last token tile to finish also runs the permutation
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(a.meta + kMetaRouteCounter, 1);
-    s_last = (prev == (int)gridDim.x - 1);
-    if (s_last) a.meta[kMetaRouteCounter] = 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  block_permute_small(a);
-}
-
-// Few-token path: CTA = 16 tokens x 8 experts, 8 warps splitting K.  The
-// CTA's 8 proj rows, the scale vector and the tile's x rows are brought into
-// shared memory by bulk copies (one round trip per K chunk of up to 2816
-// elements), then every operand comes from shared memory.
-constexpr int kStageChunk = 2816;  // K elements staged per chunk
-
-struct RouteStage {
-  uint16_t proj[8][kStageChunk];
-  uint16_t scale[kStageChunk];
-  uint16_t x[16][kStageChunk];
-  uint64_t bar;
-};
-
-__global__ void __launch_bounds__(kRouteThreads) route_staged_kernel(RouteArgs a) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  RouteStage& st = *reinterpret_cast<RouteStage*>(smem_raw);
-  __shared__ float4 s_red[kRouteThreads / 32][32];
-  __shared__ float s_ss[kRouteThreads / 32][16];
-  __shared__ int s_last;
-  __shared__ int s_abort;
-
-  const int tile = blockIdx.x, eg = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-  const int e_base = eg * 8;
-  const int tok0 = tile * 16;
-  const int ntok = min(16, a.T - tok0);
-  const int t0 = tok0 + g, t1 = t0 + 8;
-  const bool v0 = g < ntok, v1 = g + 8 < ntok;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&st.bar, 1);
-    s_abort = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  float ss0 = 0.f, ss1 = 0.f;
-  uint32_t phase = 0;
-  for (int k0 = 0; k0 < a.H; k0 += kStageChunk) {
-    const int ck = min(kStageChunk, a.H - k0);          // multiple of 128
-    const uint32_t row_bytes = (uint32_t)ck * 2;
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(&st.bar, row_bytes * (8 + 1 + ntok));
-      for (int r = 0; r < 8; ++r)
-        bulk_g2s(st.proj[r], a.proj + (size_t)(e_base + r) * a.H + k0, row_bytes, &st.bar);
-      bulk_g2s(st.scale, a.scale + k0, row_bytes, &st.bar);
-      for (int r = 0; r < ntok; ++r)
-        bulk_g2s(st.x[r], a.x + (size_t)(tok0 + r) * a.H + k0, row_bytes, &st.bar);
-    }
-    if (!mbar_wait_bounded(&st.bar, phase)) {
-      record_status(a.status, kStatusTimeout);
-      atomicExch(&s_abort, 1);
-    }
-    phase ^= 1;
-    __syncthreads();
-    if (s_abort) {
-      // drain (bounded) the copies of this chunk before leaving
-      if (threadIdx.x == 0) mbar_wait_bounded(&st.bar, phase ^ 1, kAbortDrainNs);
-      return;
-    }
-    const int nseg = ck / kSegK;
-    for (int seg = warp; seg < nseg; seg += kRouteThreads / 32) {
-#pragma unroll
-      for (int sub = 0; sub < 4; ++sub) {
-        const int k = seg * kSegK + 32 * q + 8 * sub;   // within the chunk
-        const uint4 zero = make_uint4(0, 0, 0, 0);
-        const uint4 xa = v0 ? lds_v4(&st.x[g][k]) : zero;
-        const uint4 xb = v1 ? lds_v4(&st.x[g + 8][k]) : zero;
-        const uint4 sc = lds_v4(&st.scale[k]);
-        const uint4 bw = lds_v4(&st.proj[g][k]);
-        const uint32_t xaw[4] = {xa.x, xa.y, xa.z, xa.w}, xbw[4] = {xb.x, xb.y, xb.z, xb.w};
-        const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
-        uint32_t hi_a[4], lo_a[4], hi_b[4], lo_b[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float s0 = bf16_bits_to_f32(scw[w] & 0xFFFFu), s1 = bf16_bits_to_f32(scw[w] >> 16);
-          const float xa0 = bf16_bits_to_f32(xaw[w] & 0xFFFFu), xa1 = bf16_bits_to_f32(xaw[w] >> 16);
-          const float xb0 = bf16_bits_to_f32(xbw[w] & 0xFFFFu), xb1 = bf16_bits_to_f32(xbw[w] >> 16);
-          split_hi_lo(__fmul_rn(xa0, s0), __fmul_rn(xa1, s1), hi_a[w], lo_a[w]);
-          split_hi_lo(__fmul_rn(xb0, s0), __fmul_rn(xb1, s1), hi_b[w], lo_b[w]);
-          ss0 = __fmaf_rn(xa0, xa0, ss0);
-          ss0 = __fmaf_rn(xa1, xa1, ss0);
-          ss1 = __fmaf_rn(xb0, xb0, ss1);
-          ss1 = __fmaf_rn(xb1, xb1, ss1);
-        }
-        const uint32_t Ah0[4] = {hi_a[0], hi_b[0], hi_a[1], hi_b[1]};
-        const uint32_t Al0[4] = {lo_a[0], lo_b[0], lo_a[1], lo_b[1]};
-        const uint32_t Ah1[4] = {hi_a[2], hi_b[2], hi_a[3], hi_b[3]};
-        const uint32_t Al1[4] = {lo_a[2], lo_b[2], lo_a[3], lo_b[3]};
-        mma_bf16_16816(acc, Ah0, bw.x, bw.y);
-        mma_bf16_16816(acc, Al0, bw.x, bw.y);
-        mma_bf16_16816(acc, Ah1, bw.z, bw.w);
-        mma_bf16_16816(acc, Al1, bw.z, bw.w);
-      }
-    }
-    __syncthreads();  // the chunk buffers are reused by the next chunk
-  }
-
-  ss0 += __shfl_xor_sync(0xffffffffu, ss0, 1);
-  ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
-  ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
-  ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
-  if (q == 0) {
-    s_ss[warp][g] = ss0;
-    s_ss[warp][g + 8] = ss1;
-  }
-  s_red[warp][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  __syncthreads();
-  if (warp == 0) {
-    float ssa = 0.f, ssb = 0.f;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w = 0; w < kRouteThreads / 32; ++w) {
-      ssa += s_ss[w][g];
-      ssb += s_ss[w][g + 8];
-      const float4 o = s_red[w][lane];
-      v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
-    }
-    const float fa = (1.0f / sqrtf(ssa / (float)a.H + a.eps)) * a.inv_sqrt_h;
-    const float fb = (1.0f / sqrtf(ssb / (float)a.H + a.eps)) * a.inv_sqrt_h;
-    const int e = e_base + 2 * q;
-    const float b0 = a.bias ? a.bias[e] : 0.f, b1 = a.bias ? a.bias[e + 1] : 0.f;
-    if (v0) *reinterpret_cast<float2*>(a.logits + (size_t)t0 * kE + e) = make_float2(v.x * fa + b0, v.y * fa + b1);
-    if (v1) *reinterpret_cast<float2*>(a.logits + (size_t)t1 * kE + e) = make_float2(v.z * fb + b0, v.w * fb + b1);
-  }
-
-  // the last of the 16 CTAs of this token tile runs softmax / top-8
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(a.tile_counter + tile, 1);
-    s_last = (prev == kE / 8 - 1);
-    if (s_last) a.tile_counter[tile] = 0;  // leave the counter zero for the next call
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  float pesv[4], bv_unused[4];
-  load_expert_consts(a, pesv, bv_unused);
-  for (int j = 0; j < 2; ++j) {
-    const int t = tok0 + warp * 2 + j;
-    if (t >= a.T) break;
-    float lg[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) lg[i] = __ldcg(a.logits + (size_t)t * kE + lane + 32 * i);
-    finish_token(a, t, lg, pesv);
-  }
-  if (a.meta == nullptr) return;
-  // few tokens: the last token tile to finish also runs the permutation
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(a.meta + kMetaRouteCounter, 1);
-    s_last = (prev == (int)gridDim.x - 1);
-    if (s_last) a.meta[kMetaRouteCounter] = 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  block_permute_small(a);
 }
 
 // ------------------------------------------------------------------------
@@ -917,16 +592,9 @@ __global__ void __launch_bounds__(kRwThreads, 1)
 }
 
 cudaError_t launch_route_wide(const RouteArgs& a, cudaStream_t st) {
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
   const int smem = (int)sizeof(RwSmem) + 1024;
-  if (configured_dev != dev) {
-    err = cudaFuncSetAttribute(route_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-    configured_dev = dev;
-  }
+  cudaError_t err = configure_kernel_once((const void*)route_wide_kernel, smem);
+  if (err != cudaSuccess) return err;
   CUtensorMap tm_proj, tm_x;
   if (!encode_tma_2d(&tm_proj, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.proj, (uint64_t)a.H, kE, (uint64_t)a.H * 2, 64, kE,
                      CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -939,18 +607,9 @@ cudaError_t launch_route_wide(const RouteArgs& a, cudaStream_t st) {
 
 template <int TOK>
 cudaError_t launch_route_cluster(const RouteArgs& a, cudaStream_t st) {
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
   const int smem = (int)sizeof(RcSmem<TOK>) + 1024;  // + alignment slack
-  if (configured_dev != dev) {
-    err = cudaFuncSetAttribute(route_cluster_kernel<TOK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err == cudaSuccess)
-      err = cudaFuncSetAttribute(route_cluster_kernel<TOK>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (err != cudaSuccess) return err;
-    configured_dev = dev;
-  }
+  cudaError_t err = configure_kernel_once((const void*)route_cluster_kernel<TOK>, smem, true);
+  if (err != cudaSuccess) return err;
   const int nr = a.H / kRcK;
   CUtensorMap tm_proj, tm_x;
   if (!encode_tma_2d(&tm_proj, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.proj, (uint64_t)a.H, kE, (uint64_t)a.H * 2, 64, kE,
@@ -978,27 +637,10 @@ static_assert(sizeof(RcSmem<16>) + 1024 + 8192 <= 232448, "shared memory budget 
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
-  // few tokens and hidden sizes of 8 to 16 slices of 256: one cluster per 16 tokens
-  if (a.few_tokens && a.H % kRcK == 0 && a.H / kRcK >= kRcMinRanks && a.H / kRcK <= kRcMaxRanks)
-    return launch_route_cluster<16>(a, st);
-  // many tokens: 32 tokens per CTA over the whole K
-  if (!a.few_tokens && a.H % 64 == 0) return launch_route_wide(a, st);
-  if (a.few_tokens) {
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
-    const int smem = (int)sizeof(RouteStage);
-    if (configured_dev != dev) {
-      err = cudaFuncSetAttribute(route_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (err != cudaSuccess) return err;
-      configured_dev = dev;
-    }
-    route_staged_kernel<<<dim3((a.T + 15) / 16, kE / 8), kRouteThreads, smem, st>>>(a);
-  } else {
-    route_kernel<128><<<dim3((a.T + 15) / 16, 1), kRouteThreads, 0, st>>>(a);
-  }
-  return cudaGetLastError();
+  // the C ABI admits hidden sizes of 8 to 16 slices of 256 (clusters of 8 to 16 CTAs)
+  if (a.H % kRcK != 0 || a.H / kRcK < kRcMinRanks || a.H / kRcK > kRcMaxRanks) return cudaErrorInvalidValue;
+  // few tokens: one cluster per 16 tokens; many tokens: 32 tokens per CTA over the whole K
+  return a.few_tokens ? launch_route_cluster<16>(a, st) : launch_route_wide(a, st);
 }
 
 }  // namespace nvfp4moe

@@ -224,15 +224,26 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
   // the epilogue's global reads, issued now so their latency hides behind the
   // unit's stages: the expert's global scale and (down) the routing weight of
   // each of this lane's token columns
+  // the expert's global scale, each token column's prescale exponent and
+  // (down) its routing weight, folded into one factor per column:
+  //   gate_up: G_gu * 2^(e - 15) (undoes the activation prescale)
+  //   down:    w * G_d * 2^(2 h_exp(e)) (undoes the hidden prescale)
   const float G = KIND == kGateUp ? __ldg(p.gu_g + U.e) : __ldg(p.dn_g + U.e);
-  float wgt[NNT][2];
+  float wgt[NNT][2];  // gate_up: G_gu * 2^(e - 15); down: w * G_d * 2^(2 h_exp(e))
+  float hsc[NNT][2];  // gate_up: 2^(-2 h_exp(e))
 #pragma unroll
   for (int nt = 0; nt < NNT; ++nt)
 #pragma unroll
     for (int c2 = 0; c2 < 2; ++c2) {
       const int n = nt * 8 + 2 * q + c2;
-      wgt[nt][c2] = 0.f;
-      if (KIND == kDown && n < U.nvalid) wgt[nt][c2] = __ldg(p.wts + __ldg(p.sorted_slot + U.off + U.tg * kUTok + n));
+      const int pos = U.off + U.tg * kUTok + n;
+      const int e = n < U.nvalid ? __ldg(p.xexp + pos) : 0;
+      if (KIND == kGateUp) {
+        wgt[nt][c2] = G * exp2i(e - 15);
+        hsc[nt][c2] = exp2i(-2 * h_exp(e));
+      } else {
+        wgt[nt][c2] = n < U.nvalid ? __ldg(p.wts + __ldg(p.sorted_slot + pos)) * G * exp2i(2 * h_exp(e)) : 0.f;
+      }
     }
   float acc[NNT][CH][4];
 #pragma unroll
@@ -266,6 +277,7 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
   }
 
   // ------------------------------------------------------------ epilogue
+  bool over = false;
 #pragma unroll
   for (int nt = 0; nt < NNT; ++nt) {
     float v[4];
@@ -283,15 +295,18 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
       const int pos = U.off + U.tg * kUTok + n;
       if (KIND == kGateUp) {
         const int unit = U.j * 64 + 8 * wq + g;
-        p.h[(size_t)pos * kI + unit] = f32_to_f16_sat(gelu_tanh(G * v[c2]) * (G * v[2 + c2]));
+        const float gs = wgt[nt][c2];
+        p.h[(size_t)pos * kI + unit] = f32_to_f16_sat(gelu_tanh(gs * v[c2]) * (gs * v[2 + c2]) * hsc[nt][c2], over);
       } else {
-        const float wg = wgt[nt][c2] * G;
+        const float wg = wgt[nt][c2];
         const int row0 = U.j * kURows + 16 * wq + g;
         p.obuf[(size_t)pos * kH + row0] = v[c2] * wg;
         p.obuf[(size_t)pos * kH + row0 + 8] = v[2 + c2] * wg;
       }
     }
   }
+  if (KIND == kGateUp && __any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0)
+    record_status(p.status, kStatusRange);
   return true;
 }
 
@@ -437,16 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int KIND>
 cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t st) {
   using C = SCfg<KIND>;
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
   const int smem = (int)sizeof(SSmem) + 1024;  // + alignment slack
-  if (configured_dev != dev) {
-    err = cudaFuncSetAttribute(stream_gemv_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-    configured_dev = dev;
-  }
+  cudaError_t err = configure_kernel_once((const void*)stream_gemv_kernel<KIND>, smem);
+  if (err != cudaSuccess) return err;
   CUtensorMap tm_code;
   bool ok;
   if (KIND == kGateUp) {
@@ -476,7 +484,7 @@ cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t st) {
   }
   if (!ok) return cudaErrorInvalidValue;
   int sms = 0;
-  err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  err = sm_count(&sms);
   if (err != cudaSuccess) return err;
   stream_gemv_kernel<KIND><<<sms, kThreads, smem, st>>>(tm_code, tm_x8, tm_x16, a);
   return cudaGetLastError();

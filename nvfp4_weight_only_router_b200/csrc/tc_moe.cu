@@ -89,7 +89,12 @@ struct alignas(1024) MoeSmem {
   int mt_prefix[kE + 1];
   int abort_flag;
   int issued_chunks;                     // producer progress (for draining after an abort)
-  float wslot[4][NT];                    // down: routing weight x G_d per token (one copy per epilogue warp)
+  // per token column of the current tile, one copy per epilogue warp:
+  // gate_up: the token's prescale exponent e; down: routing weight x G_d x 2^(2 h_exp(e))
+  union {
+    float w;
+    int e;
+  } tokc[4][NT];
 };
 
 struct TileInfo {
@@ -366,24 +371,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int db = titer % C::ND, duse = titer / C::ND;
       const int nvalid = min(NT, ti.cnt - ti.i * NT);
       const int pos0 = ti.off + ti.i * NT;
-      if (KIND == kDown) {
-        // routing weight x G_d of each token column, in this warp's own copy
+      {
+        // per token column: its prescale exponent (gate_up) or routing weight x
+        // G_d x 2^(2 h_exp(e)) (down), in this warp's own copy; all slot ids and
+        // exponents first, then the weights: two memory round trips per tile
         __syncwarp();
-        const float G = p.dn_g[ti.e];
-        // all slot ids first, then all weights: two memory round trips per tile
         constexpr int PER = (NT + 31) / 32;
-        int slot[PER];
+        int ex[PER], slot[PER];
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
           const int n = lane + 32 * i;
-          slot[i] = n < nvalid ? __ldg(p.sorted_slot + pos0 + n) : -1;
+          ex[i] = n < nvalid ? __ldg(p.xexp + pos0 + n) : 0;
+          slot[i] = (KIND == kDown && n < nvalid) ? __ldg(p.sorted_slot + pos0 + n) : -1;
         }
-        float wv[PER];
+        if (KIND == kDown) {
+          const float G = p.dn_g[ti.e];
+          float wv[PER];
 #pragma unroll
-        for (int i = 0; i < PER; ++i) wv[i] = slot[i] >= 0 ? __ldg(p.wts + slot[i]) : 0.f;
+          for (int i = 0; i < PER; ++i) wv[i] = slot[i] >= 0 ? __ldg(p.wts + slot[i]) : 0.f;
 #pragma unroll
-        for (int i = 0; i < PER; ++i)
-          if (lane + 32 * i < NT) sm.wslot[quarter][lane + 32 * i] = wv[i] * G;
+          for (int i = 0; i < PER; ++i)
+            if (lane + 32 * i < NT) sm.tokc[quarter][lane + 32 * i].w = wv[i] * G * exp2i(2 * h_exp(ex[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < PER; ++i)
+            if (lane + 32 * i < NT) sm.tokc[quarter][lane + 32 * i].e = ex[i];
+        }
         __syncwarp();
       }
       if (!wait_or_abort(sm, &sm.d_full[db], duse & 1, p.status)) break;
@@ -397,6 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float G = p.gu_g[ti.e];
         const bool odd = L & 1;
         const int ul = lane >> 1;  // unit within the warp's 16
+        bool over = false;
         for (int cc = 0; cc * 16 < nvalid; ++cc) {
           float v[16];
           tmem_ld16(trow + cc * 16, v);
@@ -416,9 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float g = odd ? o[k + 8] : v[k];
             const float u = odd ? v[k + 8] : o[k];
             const int n = cc * 16 + (odd ? k + 8 : k);
-            reinterpret_cast<__half*>(stg)[n * 16 + ul] = f32_to_f16_sat(gelu_tanh(G * g) * (G * u));
+            // undo the activation prescale, then apply the hidden one
+            const int e = sm.tokc[quarter][n].e;
+            const float gs = G * exp2i(e - 15);
+            reinterpret_cast<__half*>(stg)[n * 16 + ul] =
+                f32_to_f16_sat(gelu_tanh(gs * g) * (gs * u) * exp2i(-2 * h_exp(e)), over);
           }
         }
+        if (__any_sync(0xffffffffu, over) && lane == 0) record_status(p.status, kStatusRange);
         __syncwarp();
         const int jbase = ti.j * 64 + quarter * 16;
         for (int idx = lane; idx < nvalid * 2; idx += 32) {
@@ -445,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nmax = min(CW, nvalid - cc * CW);
 #pragma unroll
           for (int k = 0; k < CW; ++k)
-            if (k < nmax) p.obuf[(size_t)(pos0 + cc * CW + k) * kH + row] = v[k] * sm.wslot[quarter][cc * CW + k];
+            if (k < nmax) p.obuf[(size_t)(pos0 + cc * CW + k) * kH + row] = v[k] * sm.tokc[quarter][cc * CW + k].w;
         }
       }
       tc_fence_before();
@@ -475,16 +494,9 @@ static_assert(sizeof(MoeSmem<kDown, 192>) + 1024 <= 232448, "shared memory budge
 
 template <int KIND, int NT>
 cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
-  static int configured_dev = -1;
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
   const int smem = (int)sizeof(MoeSmem<KIND, NT>) + 1024;  // + alignment slack
-  if (configured_dev != dev) {
-    err = cudaFuncSetAttribute(tc_moe_kernel<KIND, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-    configured_dev = dev;
-  }
+  cudaError_t err = configure_kernel_once((const void*)tc_moe_kernel<KIND, NT>, smem);
+  if (err != cudaSuccess) return err;
   const uint64_t S = (uint64_t)a.T * kTopK;
   CUtensorMap tm_x, tm_w;
   bool ok;
@@ -499,20 +511,25 @@ cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
   }
   if (!ok) return cudaErrorInvalidValue;
   int sms = 0;
-  err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  err = sm_count(&sms);
   if (err != cudaSuccess) return err;
   tc_moe_kernel<KIND, NT><<<sms, kThreads, smem, st>>>(tm_x, tm_w, a);
   return cudaGetLastError();
 }
 
-// xs[pos] = f16(x[token of sorted slot pos]) (saturating): the activations in
-// expert order and in the f16 of the MMA operands, so that every tile of the
-// expert GEMMs reads contiguous rows.  One warp per row: 352 16-byte chunks,
-// 11 per lane, all loads in flight before the stores.
+// xs[pos] = f16(x[t] * 2^(15 - e_t)) and xexp[pos] = e_t for the token t of
+// sorted slot pos, e_t = floor(log2 max|x[t]|) clamped to [kXExpMin,
+// kXExpMax] (e_t = 0 for a zero row): the activations in expert order and in
+// the f16 of the MMA operands, so that every tile of the expert GEMMs reads
+// contiguous rows.  The scaled row's maximum lies in [2^15, 2^16), so every
+// bf16 element down to 2^-32 of the row maximum is exact in f16.  One warp
+// per row: 352 16-byte chunks, 11 per lane, all loads in flight before the
+// stores.
 __global__ void __launch_bounds__(256) gather_sorted_kernel(const uint16_t* __restrict__ x,
                                                             const int* __restrict__ sorted_slot,
                                                             const int* __restrict__ meta, int T,
-                                                            __half* __restrict__ xs, int* status) {
+                                                            __half* __restrict__ xs, int* __restrict__ xexp,
+                                                            int* status) {
   constexpr int per_row = kH / 8;              // 352
   constexpr int per_lane = per_row / 32;       // 11
   const int S = meta[kMetaOffsets + kE];
@@ -528,15 +545,32 @@ __global__ void __launch_bounds__(256) gather_sorted_kernel(const uint16_t* __re
     uint4 v[per_lane];
 #pragma unroll
     for (int i = 0; i < per_lane; ++i) v[i] = ldg_nc_v4(src + lane + 32 * i);
+    // the row maximum of |x| as a bf16 bit pattern (monotone for finite values)
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int i = 0; i < per_lane; ++i)
+      m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu),
+                                 __vmaxu2(v[i].z & 0x7FFF7FFFu, v[i].w & 0x7FFF7FFFu)));
+    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // floor(log2 max|x|) is the unbiased exponent field (a subnormal maximum
+    // clamps to kXExpMin)
+    const int e = m == 0 ? 0 : max(kXExpMin, min(kXExpMax, (int)(m >> 7) - 127));
+    const float sc = exp2i(15 - e);
+    bool over = false;
 #pragma unroll
     for (int i = 0; i < per_lane; ++i) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       uint32_t o[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        o[k] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(w[k] & 0xFFFFu)), f32_to_f16_sat(bf16_bits_to_f32(w[k] >> 16)));
+        o[k] = pack_f16x2(f32_to_f16_sat(bf16_bits_to_f32(w[k] & 0xFFFFu) * sc, over),
+                          f32_to_f16_sat(bf16_bits_to_f32(w[k] >> 16) * sc, over));
       __stcs(dst + lane + 32 * i, make_uint4(o[0], o[1], o[2], o[3]));
     }
+    if (lane == 0) xexp[pos] = e;
+    if (__any_sync(0xffffffffu, over) && lane == 0) record_status(status, kStatusRange);
   }
 }
 
@@ -546,7 +580,7 @@ cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st) {
   const int64_t rows = (int64_t)a.T * kTopK;
   int blocks = (int)((rows + 7) / 8);
   if (blocks > 148 * 32) blocks = 148 * 32;
-  gather_sorted_kernel<<<blocks, 256, 0, st>>>(a.x, a.sorted_slot, a.meta, a.T, a.xs, a.status);
+  gather_sorted_kernel<<<blocks, 256, 0, st>>>(a.x, a.sorted_slot, a.meta, a.T, a.xs, a.xexp, a.status);
   return cudaGetLastError();
 }
 

@@ -25,7 +25,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported(capi):
     names = header_functions()
-    assert len(names) == 15
+    assert len(names) == 18
     for n in names:
         assert hasattr(capi.lib, n), n
         assert n in capi.SIGNATURES, n
@@ -38,8 +38,8 @@ def test_only_declared_symbols_are_exported(capi):
 
 
 def test_abi_version_and_status_strings(capi):
-    assert capi.nvfp4_abi_version() == 1
-    for code in range(8):
+    assert capi.nvfp4_abi_version() == 2
+    for code in range(9):
         assert capi.status_string(code)
     assert capi.status_string(0) == "ok"
 
@@ -84,7 +84,9 @@ def test_route_validation(capi):
     assert c.moe_route(P, 0, ctypes.byref(r), P, P, P, 1 << 20, None) == c.NVFP4_ERR_INVALID_ARG
     assert c.moe_route(P, 1, None, P, P, P, 1 << 20, None) == c.NVFP4_ERR_INVALID_ARG
     for bad, code in [(_router(c, E=64), c.NVFP4_ERR_UNSUPPORTED), (_router(c, k=4), c.NVFP4_ERR_UNSUPPORTED),
-                      (_router(c, H=100), c.NVFP4_ERR_UNSUPPORTED), (_router(c, eps=-1.0), c.NVFP4_ERR_INVALID_ARG),
+                      (_router(c, H=100), c.NVFP4_ERR_UNSUPPORTED), (_router(c, H=1792), c.NVFP4_ERR_UNSUPPORTED),
+                      (_router(c, H=4352), c.NVFP4_ERR_UNSUPPORTED), (_router(c, H=2880), c.NVFP4_ERR_UNSUPPORTED),
+                      (_router(c, eps=-1.0), c.NVFP4_ERR_INVALID_ARG),
                       (_router(c, ptr=4097), c.NVFP4_ERR_ALIGNMENT)]:
         assert c.moe_route(P, 1, ctypes.byref(bad), P, P, P, 1 << 20, None) == code
     assert c.moe_route(P + 2, 1, ctypes.byref(r), P, P, P, 1 << 20, None) == c.NVFP4_ERR_ALIGNMENT
@@ -109,7 +111,7 @@ def test_forward_validation_and_workspace_sizes(capi):
     assert c.moe_nvfp4_forward(P, 1, ctypes.byref(x), ctypes.byref(r), P, P + 128, ws, None) == c.NVFP4_ERR_ALIGNMENT
     v = c.moe_forward_views()
     assert c.moe_forward_workspace_views(64, ctypes.byref(x), ctypes.byref(r), ctypes.byref(v)) == 0
-    offs = [v.ids, v.weights, v.counts, v.offsets, v.sorted_slot, v.slot_pos, v.h]
+    offs = [v.ids, v.weights, v.counts, v.offsets, v.sorted_slot, v.slot_pos, v.xexp, v.h]
     assert all(o % 4 == 0 for o in offs) and max(offs) < sizes[1]
 
 
@@ -124,3 +126,39 @@ def test_residual_validation(capi):
 def test_last_cuda_error_is_a_string_before_any_failure(capi):
     # no call of this thread has failed yet: the runtime's text for success
     assert capi.lib.nvfp4_last_cuda_error().decode() == "no error"
+
+
+def test_permute_validation(capi):
+    c = capi
+    assert c.moe_permute_workspace_bytes(0) == 0
+    assert c.moe_permute_workspace_bytes(65537) == 0
+    small, big = c.moe_permute_workspace_bytes(1), c.moe_permute_workspace_bytes(65536)
+    assert 0 < small < big
+    P = 4096
+    assert c.moe_permute(None, 1, P, P, P, P, P, small, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_permute(P, 0, P, P, P, P, P, small, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_permute(P, 1, P, P + 4, P, P, P, small, None) == c.NVFP4_ERR_ALIGNMENT
+    assert c.moe_permute(P, 1, P, P, P, P, P, small - 1, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.moe_permute(P, 1, P, P, P, P, P + 16, small, None) == c.NVFP4_ERR_ALIGNMENT
+
+
+def test_selftest_validation(capi):
+    c = capi
+    P = 4096
+    ws = c.nvfp4_quantize_workspace_bytes(2, 1408, 2816)
+    assert c.nvfp4_selftest_wait_timeout(P, 2, 1408, 2816, P, P, P, P, ws, 0, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.nvfp4_selftest_wait_timeout(P, 2, 1408, 2816, P, P, P, P, ws, 1000001, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.nvfp4_selftest_wait_timeout(P, 2, 1408, 2816, P, P, P, None, ws, 1000, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.nvfp4_selftest_wait_timeout(P + 2, 2, 1408, 2816, P, P, P, P, ws, 1000, None) == c.NVFP4_ERR_ALIGNMENT
+
+
+def test_last_cuda_error_after_a_failed_call_without_a_device(capi):
+    """With no CUDA device, a valid no-allocation quantise fails in its first
+    runtime call (before any launch): the status is NVFP4_ERR_CUDA and
+    nvfp4_last_cuda_error names the runtime's error, not "no error"."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a host without a CUDA device (the call would launch on fake pointers)")
+    P = 4096
+    assert capi.nvfp4_quantize_noalloc(P, 1, 16, 32, P, P, P, None) == capi.NVFP4_ERR_CUDA
+    assert capi.lib.nvfp4_last_cuda_error().decode() != "no error"

@@ -70,23 +70,68 @@ def test_edge_values(dev, N, K):
     _assert_equal_quant(_run(bits, dev), Q.quantize(bits))
 
 
-def test_full_size_sampled_and_roundtrip(dev):
-    """[128, 1408, 2816] bf16 (the expert gate_up stack shape), built from 8
-    independently drawn experts repeated 16 times; experts from each copy
-    group are compared with the oracle, and the fp32 dequantisation of them
-    round-trips bit-exactly."""
-    base = gen.make_quant_weights(4, 8, 1408, 2816)
-    bits = np.tile(base, (16, 1, 1))
-    wd = bf16_to_dev(bits, dev)
-    q, s, g = lib.quantize(wd)
-    deq = lib.dequantize(q, s, g)
-    torch.cuda.synchronize()
+def test_full_size_workload_all_tensors(dev):
+    """The quantise workload itself: bf16 [128, 1408, 2816] ~ N(0, 0.02) with
+    0.5% x20 outliers (expert j from its own seeded stream), every one of the
+    128 tensors bit-exact against the oracle (run in a process pool), and the
+    fp32 dequantisation of four of them round-tripping bit-exactly."""
+    from tests.oracle_pool import pool, quant_expert_and_oracle
+    E, N, K = 128, 1408, 2816
+    with pool() as ex:
+        res = list(ex.map(quant_expert_and_oracle, [(4, j, N, K) for j in range(E)]))
+    w = np.stack([r[0] for r in res])
+    q, s, g = _run(w, dev)
     assert lib.device_status() == 0
-    for e in (0, 5, 63, 127):
-        want = Q.quantize_tensor(bits[e])
-        got = (q[e].cpu().numpy(), s[e].cpu().numpy(), g[e:e + 1].cpu().numpy())
-        _assert_equal_quant(got, (want[0], want[1], np.array([want[2]])))
-        d0 = Q.dequantize_f32(want[0], want[1], want[2])
-        assert np.array_equal(deq[e].cpu().numpy().view(np.uint32), d0.view(np.uint32))
-    # identical copies quantise identically
-    assert torch.equal(q[0], q[8]) and torch.equal(s[3], s[3 + 64])
+    for j, (_, q0, s0, g0) in enumerate(res):
+        assert g[j].view(np.uint32) == np.float32(g0).view(np.uint32), j
+        assert np.array_equal(s[j], s0), f"tensor {j}: {np.count_nonzero(s[j] != s0)} scale bytes differ"
+        assert np.array_equal(q[j], q0), f"tensor {j}: {np.count_nonzero(q[j] != q0)} code bytes differ"
+    qd, sd, gd = (torch.from_numpy(a).to(dev) for a in (q, s, g))
+    deq = lib.dequantize(qd, sd, gd)
+    torch.cuda.synchronize()
+    for j in (0, 5, 63, 127):
+        d0 = Q.dequantize_f32(res[j][1], res[j][2], res[j][3])
+        assert np.array_equal(deq[j].cpu().numpy().view(np.uint32), d0.view(np.uint32))
+
+
+def test_more_tensors_than_a_grid_dimension(dev):
+    """65,600 tiny tensors [1, 32] (the two-pass kernels, whose amax pass puts
+    tensors on the grid's y dimension, at most 65,535): the tensors past that
+    limit are quantised too; bit-exact on every tensor of a sample that covers
+    both sides of the limit."""
+    E = 65600
+    bits = gen.make_quant_weights(9, E, 1, 32)
+    q, s, g = _run(bits, dev)
+    assert lib.device_status() == 0
+    sample = np.r_[0:64, 65500:65600, np.random.default_rng(1).choice(E, 200, replace=False)]
+    for j in sample:
+        q0, s0, g0 = Q.quantize_tensor(bits[j])
+        assert g[j].view(np.uint32) == np.float32(g0).view(np.uint32), j
+        assert np.array_equal(s[j], s0) and np.array_equal(q[j], q0), j
+
+
+def test_timeout_selftest_then_gpu_still_answers(dev):
+    """A bounded wait that cannot complete: the single-pass quantiser's
+    cross-CTA arrival count raised past what the grid can reach, every wait
+    limited to 20 ms.  The call returns, the device status reads
+    NVFP4_ERR_TIMEOUT, and the GPU still answers: a quantise right after is
+    bit-exact against the oracle."""
+    import time
+    from nvfp4_weight_only_router_b200 import capi
+    bits = gen.make_quant_weights(13, 2, 1408, 2816)
+    w = bf16_to_dev(bits, dev)
+    q = torch.empty((2, 1408, 1408), dtype=torch.uint8, device=dev)
+    s = torch.empty((2, 1408, 176), dtype=torch.uint8, device=dev)
+    g = torch.empty((2,), dtype=torch.float32, device=dev)
+    nbytes = capi.nvfp4_quantize_workspace_bytes(2, 1408, 2816)
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    assert lib.device_status() == 0
+    t0 = time.perf_counter()
+    capi.check(capi.nvfp4_selftest_wait_timeout(w.data_ptr(), 2, 1408, 2816, q.data_ptr(), s.data_ptr(),
+                                                g.data_ptr(), ws.data_ptr(), ws.numel(), 20000,
+                                                torch.cuda.current_stream().cuda_stream))
+    assert capi.nvfp4_get_device_status(None) == capi.NVFP4_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert capi.nvfp4_get_device_status(None) == capi.NVFP4_OK   # read and cleared
+    _assert_equal_quant(_run(bits, dev), Q.quantize(bits))
+    assert lib.device_status() == 0

@@ -35,11 +35,23 @@ def test_route_prefill_zipf_bias(dev):
     assert differ.mean() < 1e-3
 
 
-def test_route_other_hidden_size(dev):
-    rt = gen.make_router(5, h=256)
+def test_route_unsupported_hidden_size(dev):
+    # hidden sizes that are not 8 to 16 slices of 256 are refused up front
+    rt = gen.make_router(5, h=640)
     drt = lib.Router.from_host(rt, dev)
-    x = gen.make_x(6, 33, 256)
-    _check(x, rt, drt, dev)
+    with pytest.raises(lib.NVFP4Error) as e:
+        lib.route(bf16_to_dev(gen.make_x(6, 3, 640), dev), drt)
+    assert e.value.status == lib.capi.NVFP4_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("T", [1, 5, 64, 256])
+def test_route_cluster_with_logit_bias(dev, T):
+    """A logit bias through the few-token cluster kernel: a random bias (the
+    Zipf bias of the prefill workload is checked at T = 4096 and at T = 64)."""
+    bias = np.random.default_rng(T).normal(0, 0.05, 128).astype(np.float32) if T != 64 else gen.zipf_bias(7)
+    rt = gen.make_router(1, bias=bias)
+    drt = lib.Router.from_host(rt, dev)
+    _check(gen.make_x(300 + T, T), rt, drt, dev)
 
 
 def test_route_ties_pick_lower_id(dev):
@@ -52,11 +64,10 @@ def test_route_ties_pick_lower_id(dev):
     assert (ids.cpu().numpy() == np.arange(8)[None, :]).all()
 
 
-@pytest.mark.parametrize("h,T", [(2048, 3), (2048, 40), (4096, 17), (640, 300), (384, 20), (256, 600)])
+@pytest.mark.parametrize("h,T", [(2048, 3), (2048, 40), (4096, 17), (2048, 300), (4096, 600), (3072, 257)])
 def test_route_hidden_sizes_all_paths(dev, h, T):
-    # clusters of 8 and 16 CTAs (h = 2048, 4096), the wide kernel with an odd
-    # number of 64-wide K blocks (h = 640, T > 256), and the fallbacks for hidden
-    # sizes that are not multiples of 256 (few tokens) or too small for a cluster
+    # clusters of 8, 12 and 16 CTAs (h = 2048, 3072, 4096; T <= 256) and the
+    # wide kernel (T > 256) at other hidden sizes than the layer's
     rt = gen.make_router(20 + h, h=h)
     drt = lib.Router.from_host(rt, dev)
     x = gen.make_x(21 + T, T, h)

@@ -198,3 +198,78 @@ def test_ids_override_uses_given_ids():
     y1 = M.forward(x, ex, rt)
     y2 = M.forward(x, ex, rt, ids_override=swapped)
     assert np.allclose(y1, y2, rtol=1e-12, atol=1e-18)
+
+
+# ------------------------------------------------------------- chain link pin
+def _nearest_bf16(v: np.ndarray) -> np.ndarray:
+    """The bf16 value nearest to each fp64 value (ties to the even mantissa),
+    found among torch's bf16 neighbours: torch rounds through fp32, so its
+    result may be one ulp off, and the nearest of it and its two neighbours is
+    the correctly rounded value."""
+    b = torch.from_numpy(v).float().to(torch.bfloat16)
+    cands = torch.stack([torch.nextafter(b, torch.full_like(b, -np.inf)), b,
+                         torch.nextafter(b, torch.full_like(b, np.inf))]).double().numpy()
+    bits = torch.stack([torch.nextafter(b, torch.full_like(b, -np.inf)), b,
+                        torch.nextafter(b, torch.full_like(b, np.inf))]).view(torch.int16).numpy()
+    d = np.abs(cands - v[None])
+    best = d.min(0)
+    tie_ok = (d == best[None]) & ((bits & 1) == 0)
+    pick = np.where(tie_ok.any(0), np.argmax(tie_ok, 0), np.argmin(d, 0))
+    return np.take_along_axis(cands, pick[None], 0)[0]
+
+
+def test_residual_rmsnorm_vs_torch_rms_norm():
+    rng = np.random.default_rng(21)
+    H = 96
+    res = rng.standard_normal((6, H)) * np.array([1e-3, 1.0, 1e3, 5.0, 1e-6, 1e5])[:, None]
+    y = gen.bf16_bits(rng.standard_normal((6, H)).astype(np.float32) * 0.01)
+    res2, xb = M.residual_rmsnorm(res, y, eps=1e-6)
+    y_t = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).double()
+    want_res = torch.from_numpy(res) + y_t               # the residual takes y first
+    assert np.array_equal(res2, want_res.numpy())
+    want_x = TF.rms_norm(want_res, (H,), eps=1e-6).numpy()   # eps inside the square root
+    assert np.array_equal(F.bf16_to_f64(xb), _nearest_bf16(want_x))
+
+
+def test_residual_rmsnorm_constant_row_closed_form():
+    c = 0.75
+    res = np.full((1, 64), c)
+    y = np.zeros((1, 64), np.uint16)                     # +0.0 in bf16
+    res2, xb = M.residual_rmsnorm(res, y, eps=0.25)
+    assert np.all(res2 == c)
+    # x = c / sqrt(c^2 + eps) = 0.75 / sqrt(0.8125) = 0.83205..., nearest bf16 0.83203125
+    assert np.all(F.bf16_to_f64(xb) == 0.83203125)
+
+
+# ---------------------------------------------------------- gated hidden pin
+def _brute_force_hidden(x_bits, ex, e):
+    """Pure-Python h = gelu_tanh(gate) * up of expert e for each row of x, with
+    the weights decoded element by element (E2M1 x E4M3 x global)."""
+    T, H = x_bits.shape
+    I = ex.I
+    e2m1 = [F.e2m1_decode(c).item() for c in range(16)]
+    e4m3 = [F.e4m3_decode(c).item() for c in range(256)]
+
+    def wgu(n, kk):
+        byte = int(ex.gate_up_q[e][n, kk // 2])
+        code = byte & 0xF if kk % 2 == 0 else byte >> 4
+        return e2m1[code] * e4m3[int(ex.gate_up_s[e][n, kk // 16])] * float(ex.gate_up_g[e])
+
+    out = []
+    for t in range(T):
+        xt = [F.bf16_to_f64(x_bits[t, kk]).item() for kk in range(H)]
+        gate = [sum(wgu(n, kk) * xt[kk] for kk in range(H)) for n in range(I)]
+        up = [sum(wgu(I + n, kk) * xt[kk] for kk in range(H)) for n in range(I)]
+        out.append([0.5 * g * (1 + math.tanh(math.sqrt(2 / math.pi) * (g + 0.044715 * g ** 3))) * u
+                    for g, u in zip(gate, up)])
+    return np.array(out)
+
+
+@pytest.mark.parametrize("e", [0, 3])
+def test_expert_hidden_vs_pure_python(e):
+    x, ex, _ = tiny(seed=15, T=3)
+    wgu, _ = M.expert_dense(ex, e)
+    got = M.expert_hidden(F.bf16_to_f64(x), wgu)
+    want = _brute_force_hidden(x, ex, e)
+    assert got.shape == (3, I_T)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-14 * np.abs(want).max())

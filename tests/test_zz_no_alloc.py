@@ -39,12 +39,18 @@ def _quantize_both(capi, w_bits, dev):
 
 def test_noalloc_matches_workspace_entry_point_twice(dev):
     from nvfp4_weight_only_router_b200 import capi
+    from oracle import quantize as Q
     # two calls in a row with different inputs (and a different tensor count,
-    # so stale scratch from the first call would show up in the second)
+    # so stale scratch from the first call would show up in the second); each
+    # result also against the oracle directly
     for seed, shape in ((21, (6, 96, 512)), (22, (3, 1408, 2816))):
-        ref, got = _quantize_both(capi, gen.make_quant_weights(seed, *shape), dev)
+        bits = gen.make_quant_weights(seed, *shape)
+        ref, got = _quantize_both(capi, bits, dev)
         for a, b in zip(ref, got):
             assert torch.equal(a, b)
+        q0, s0, g0 = Q.quantize(bits)
+        assert np.array_equal(got[0].cpu().numpy(), q0) and np.array_equal(got[1].cpu().numpy(), s0)
+        assert np.array_equal(got[2].cpu().numpy().view(np.uint32), g0.view(np.uint32))
     assert capi.nvfp4_get_device_status(None) == 0
 
 
