@@ -2,7 +2,8 @@
 """Benchmark of the NVFP4 weight-only MoE branch on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode64|decode1|prefill4096|stack30|quantize]
+                    [--workload decode64|decode1|dense1|prefill4096|block64|block4096|
+                                stack30|quantize]
 
 A step is one pass of the whole hot path -- route, permute, gate_up + GELU,
 down, combine -- over one batch of synthetic tokens (the default workload:
@@ -72,6 +73,12 @@ WORKLOADS = {
     "decode1": {"T": 1, "layers": 1, "zipf": False, "desc": "one MoE layer, decode T=1"},
     "prefill4096": {"T": 4096, "layers": 1, "zipf": True,
                     "desc": "one MoE layer, prefill T=4096, Zipf(1.1)-skewed router bias"},
+    "dense1": {"T": 1, "layers": 1, "zipf": False, "dense": True,
+               "desc": "one MoE layer, decode T=1, dense over-read: all 128 experts per token (ablation)"},
+    "block64": {"T": 64, "layers": 1, "zipf": False, "block": True,
+                "desc": "full MoE block (dense MLP 2112 || NVFP4 experts, norms, layer scalar), decode T=64"},
+    "block4096": {"T": 4096, "layers": 1, "zipf": True, "block": True,
+                  "desc": "full MoE block, prefill T=4096, Zipf(1.1)-skewed router bias"},
     "stack30": {"T": 8, "layers": 30, "zipf": False,
                 "desc": "30 independently seeded MoE layers chained x+=moe(rmsnorm(x)), T=8"},
     "quantize": {"T": 0, "layers": 0, "zipf": False,
@@ -165,7 +172,15 @@ class OracleSample:
         self.ex = gen.make_experts(0 if wl["layers"] == 1 else 100)
         self.rt = gen.make_router(1, bias=gen.zipf_bias(7) if wl["zipf"] else None)
         self.x = gen.make_x(10_000, max(wl["T"], tokens))[:tokens]
-        self.what = f"oracle fp64 forward of {tokens} of the workload's tokens through one layer"
+        self.block = None
+        if wl.get("block"):
+            from oracle import block as B
+            b = gen.make_block(200)
+            self.block = B.BlockParams(self.ex, self.rt, b.dense_gate, b.dense_up, b.dense_down, b.pre_ff_norm,
+                                       b.post_ff_norm_1, b.pre_ff_norm_2, b.post_ff_norm_2, b.post_ff_norm,
+                                       b.layer_scalar)
+        self.what = (f"oracle fp64 forward of {tokens} of the workload's tokens through one "
+                     + ("full block" if self.block else "layer"))
 
     def run(self):
         """Returns (value, unit, seconds)."""
@@ -177,7 +192,11 @@ class OracleSample:
             dt = time.perf_counter() - t0
             nbytes = self.w.nbytes + self.w.nbytes // 4 + self.w.nbytes // 16 + 4
             return nbytes / dt / 1e9, "GB/s", dt
-        M.forward(self.x, self.ex, self.rt)
+        if self.block is not None:
+            from oracle import block as B
+            B.forward(self.x, self.block)
+        else:
+            M.forward(self.x, self.ex, self.rt)
         dt = time.perf_counter() - t0
         return self.tokens / dt, "tokens/s", dt
 
@@ -312,7 +331,11 @@ def measure(ctx, workload, args, cpu_baseline=True):
         for sd in seeds:
             rt = gen.make_router(1 if wl["layers"] == 1 else 1000 + sd,
                                  bias=gen.zipf_bias(7) if wl["zipf"] else None)
-            layers.append(lib.MoeLayer(ctx.experts(sd), lib.Router.from_host(rt, dev), max_tokens=T))
+            if wl.get("block"):
+                parts = lib.DenseParts.from_host(gen.make_block(200), dev)
+                layers.append(lib.MoeBlock(ctx.experts(sd), lib.Router.from_host(rt, dev), parts, max_tokens=T))
+            else:
+                layers.append(lib.MoeLayer(ctx.experts(sd), lib.Router.from_host(rt, dev), max_tokens=T))
         xs_host = np.stack([gen.make_x(replica_x_seed(rank, n_pool, i), T) for i in range(n_pool)])
         x_pool = _bf(xs_host).to(dev)
         x_pin = _bf(xs_host).pin_memory()
@@ -324,7 +347,11 @@ def measure(ctx, workload, args, cpu_baseline=True):
 
         def fwd_layer(layer, xin, yout, profiled):
             st = torch.cuda.current_stream().cuda_stream
-            if profiled:
+            if wl.get("dense"):
+                layer.forward_dense_into(xin, yout)
+            elif wl.get("block"):
+                layer.forward_into(xin, yout)
+            elif profiled:
                 arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
                 capi.check(capi.moe_nvfp4_forward_profiled(
                     xin.data_ptr(), T, ctypes.byref(layer._xs), ctypes.byref(layer._rs), yout.data_ptr(),
@@ -376,6 +403,12 @@ def measure(ctx, workload, args, cpu_baseline=True):
         # permutation kernels), gather, gate_up, down, combine; plus the
         # chain's rmsnorm kernels
         per_layer = 5 if T * 8 <= 1024 else 7
+        if wl.get("dense"):
+            per_layer = 6  # route, dense permutation, gather, gate_up, down, combine
+        if wl.get("block"):
+            # prenorm, the routed branch without its combine, dense gate_up,
+            # GELU, dense down, the block's final kernel
+            per_layer = (4 if T * 8 <= 1024 else 6) + 5
         kernels_per_step = per_layer * len(layers) + (len(layers) + 1 if len(layers) > 1 else 0)
 
     # -------- warm-up (at least W steps and at least --min-warmup-s, so the clock sampler sees load)
@@ -402,8 +435,10 @@ def measure(ctx, workload, args, cpu_baseline=True):
         end.record()
         torch.cuda.synchronize()
         step_ms.append(start.elapsed_time(end))
-        if workload != "quantize":
+        if workload != "quantize" and not wl.get("block"):
             act_counts.append(int((layers[0].views(T)["counts"] > 0).sum().item()))
+        elif wl.get("block"):
+            act_counts.append(int(torch.unique(layers[0].ids(T)).numel()))
     torch.cuda.synchronize()
     # phase breakdown (and the dominant kernel's duration for the roofline):
     # the same K steps again, each replaying the graph whose event-record
@@ -411,6 +446,8 @@ def measure(ctx, workload, args, cpu_baseline=True):
     prof_ms = []
     if workload != "quantize":
         for k in range(args.steps):
+            if wl.get("dense") or wl.get("block"):
+                break  # these variants record no phase events
             ctx.flush.zero_()
             prepare(k)
             start.record()
@@ -477,18 +514,40 @@ def measure(ctx, workload, args, cpu_baseline=True):
     else:
         value = job_rate(T, world, args.steps, total_ms)
         unit = "tokens/s"
-        ph = np.array(phase_ms)  # [steps, 5]: route, permute, gate_up, down, combine
+        ph = np.array(phase_ms) if phase_ms else np.full((1, 5), np.nan)  # route, permute, gate_up, down, combine
         n_act = np.array(act_counts, np.float64)
+        if wl.get("dense"):
+            n_act = np.full_like(n_act, 128.0)  # every expert is read
         S = T * 8
         gu_bytes = n_act * GU_EXPERT_BYTES + T * 2816 * 2 + S * 704 * 2
         gu_flops = 2.0 * S * 1408 * 2816
         gu_ms = ph[:, 2]
-        if T >= 1024:
+        dense_bytes = 3 * 2816 * 2112 * 2
+        dense_flops = 2.0 * T * 3 * 2816 * 2112
+        if wl.get("block") and T >= 1024:
+            flops = 2.0 * S * (1408 * 2816 + 2816 * 704) + dense_flops
+            ach = flops / (ms_per_step / 1e3) / 1e12
+            roof = {"bound": "tensor", "kernel": "whole block step (experts + dense MLP, no phase split)",
+                    "achieved": ach, "peak": ctx.tc_peak, "unit": "TFLOP/s", "traffic": traffic,
+                    "peak_kind": ctx.peak_kind + " burst bf16", "algorithmic_per_launch": flops}
+        elif wl.get("block"):
+            nbytes = (n_act * EXPERT_BYTES + ROUTER_BYTES + dense_bytes + 2 * T * 2816 * 2).mean()
+            ach = nbytes / (ms_per_step / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": "whole block step (experts + dense MLP, no phase split)",
+                    "achieved": ach, "peak": ctx.hbm_peak, "unit": "GB/s", "traffic": traffic,
+                    "peak_kind": ctx.peak_kind, "algorithmic_per_launch": float(nbytes)}
+        elif T >= 1024:
             # a sub-millisecond kernel timed between L2 flushes: the burst peak
             ach = gu_flops / (gu_ms.mean() / 1e3) / 1e12
             roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM + GELU (tcgen05)", "achieved": ach,
                     "peak": ctx.tc_peak, "unit": "TFLOP/s", "traffic": traffic,
                     "peak_kind": ctx.peak_kind + " burst bf16", "algorithmic_per_launch": gu_flops}
+        elif wl.get("dense"):
+            # no phase split: the whole step's algorithmic bytes (all 128 experts)
+            ach = (n_act * EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2).mean() / (ms_per_step / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": "whole dense over-read step (all experts)", "achieved": ach,
+                    "peak": ctx.hbm_peak, "unit": "GB/s", "traffic": traffic, "peak_kind": ctx.peak_kind,
+                    "algorithmic_per_launch": float((n_act * EXPERT_BYTES).mean())}
         else:
             ach = gu_bytes.sum() / (gu_ms.sum() / 1e3) / 1e9
             roof = {"bound": "hbm", "kernel": "gate_up grouped GEMV + GELU", "achieved": ach,
@@ -498,9 +557,9 @@ def measure(ctx, workload, args, cpu_baseline=True):
         roof["frac"] = roof["achieved"] / roof["peak"]
         step_bytes = n_act * EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2
         extra = {
-            "phase_ms_mean": dict(zip(["route", "permute", "gate_up", "down", "combine"],
-                                      [float(v) for v in ph.mean(0)])),
-            "ms_per_step_with_phase_events": float(np.mean(prof_ms)),
+            "phase_ms_mean": None if (wl.get("dense") or wl.get("block")) else dict(zip(["route", "permute", "gate_up", "down", "combine"],
+                                                                 [float(v) for v in ph.mean(0)])),
+            "ms_per_step_with_phase_events": float(np.mean(prof_ms)) if prof_ms else None,
             "active_experts_mean": float(n_act.mean()),
             # whole-step algorithmic bytes (active experts + router + x + y) per second
             "step_hbm_gbs": float(step_bytes.mean() * wl["layers"] / (ms_per_step / 1e3) / 1e9),

@@ -208,6 +208,24 @@ NVFP4MOE_API nvfp4_status moe_nvfp4_forward(const void* x_dev, int32_t T, const 
                                const moe_router* router, void* y_dev,
                                void* ws_dev, size_t ws_bytes, void* stream);
 
+/* moe_nvfp4_forward_dense: the same output as moe_nvfp4_forward computed the
+ * way a runtime without a gather kernel does it ("Gemma 4 26B-A4B (MoE) -
+ * Core AI", "Compression recipe": without the gather kernel the sparse
+ * branch becomes a dense matmul that reads all 128 experts every token, a 16x
+ * over-read; "Performance": 140 vs 39 tok/s for another MoE through its
+ * gather kernel and as the dense over-read).  Every token goes through every
+ * expert, each expert's output weighted by the token's routing weight for it
+ * (0 for the 120 experts the router did not select), so all 128 experts'
+ * weights are read for any T.  An ablation for measuring the gather's
+ * advantage, not a path to deploy.  Same arguments and layouts as
+ * moe_nvfp4_forward; requires 1 <= T <= 256.  Workspace:
+ * moe_forward_dense_workspace_bytes(T, experts, router) bytes. */
+NVFP4MOE_API size_t moe_forward_dense_workspace_bytes(int32_t T, const moe_experts* experts,
+                                                      const moe_router* router);
+NVFP4MOE_API nvfp4_status moe_nvfp4_forward_dense(const void* x_dev, int32_t T, const moe_experts* experts,
+                                                  const moe_router* router, void* y_dev,
+                                                  void* ws_dev, size_t ws_bytes, void* stream);
+
 /* moe_nvfp4_forward_profiled: moe_nvfp4_forward that also records CUDA
  * events between its phases on `stream`.  phase_events points to 6 cudaEvent_t
  * (passed as void*; a NULL entry is skipped): [0] before the first kernel,
@@ -234,6 +252,45 @@ typedef struct {
 } moe_forward_views;
 NVFP4MOE_API nvfp4_status moe_forward_workspace_views(int32_t T, const moe_experts* experts,
                                          const moe_router* router, moe_forward_views* out);
+
+/* ---------------------------------------------------------------------------
+ * moe_block_forward: the full feed-forward half of a Gemma-4-26B-A4B decoder
+ * layer ("Gemma 4 26B-A4B (MoE) - Core AI", the layer dataflow listing): a
+ * dense GELU-gated MLP (intermediate 2112, "Architecture" table; bf16
+ * weights, "Gemma-4-26B-A4B-NVFP4-mlx", "Quantization recipe") in parallel
+ * with the NVFP4 sparse branch,
+ *   h   = mlp(pre_ff_norm(x))                 h1 = post_ff_norm_1(h)
+ *   ids, w = router(x)                        (the RAW residual)
+ *   h2  = post_ff_norm_2(sum_k w_k expert_{ids_k}(pre_ff_norm_2(x)))
+ *   y   = (x + post_ff_norm(h1 + h2)) * layer_scalar
+ * Each norm is x / sqrt(mean(x^2) + eps) * weight (fp32).  The two MLP inputs
+ * are rounded to bf16 (the modules' bf16 activations); the dense MLP runs on
+ * the tensor cores with bf16 operands and fp32 accumulation, its gated
+ * hidden entering the down projection as an exact bf16 high + low pair; the
+ * experts as in moe_nvfp4_forward; all later steps in fp32; y is rounded
+ * once to bf16.
+ *   x_dev bf16 [T, H] (in: the post-attention hidden), y_dev bf16 [T, H] (out)
+ * Requires 1 <= T <= 8192, the experts and router of moe_nvfp4_forward,
+ * dense_I == 2112.  Workspace: moe_block_workspace_bytes(T, block) bytes.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  moe_experts experts;
+  moe_router router;
+  const void* dense_gate;      /* bf16 [dense_I, H] */
+  const void* dense_up;        /* bf16 [dense_I, H] */
+  const void* dense_down;      /* bf16 [H, dense_I] */
+  const void* pre_ff_norm;     /* bf16 [H] pre_feedforward_layernorm */
+  const void* post_ff_norm_1;  /* bf16 [H] post_feedforward_layernorm_1 */
+  const void* pre_ff_norm_2;   /* bf16 [H] pre_feedforward_layernorm_2 */
+  const void* post_ff_norm_2;  /* bf16 [H] post_feedforward_layernorm_2 */
+  const void* post_ff_norm;    /* bf16 [H] post_feedforward_layernorm */
+  const void* layer_scalar;    /* bf16 [1] */
+  int32_t dense_I;             /* must be 2112 */
+  float eps;                   /* the five norms' epsilon (the pages are silent; 1e-6) */
+} moe_block;
+NVFP4MOE_API size_t moe_block_workspace_bytes(int32_t T, const moe_block* block);
+NVFP4MOE_API nvfp4_status moe_block_forward(const void* x_dev, int32_t T, const moe_block* block, void* y_dev,
+                                            void* ws_dev, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute: the token permutation of moe_nvfp4_forward on its own -- the

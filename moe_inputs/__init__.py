@@ -24,12 +24,13 @@ E = 128         # routed experts per layer
 TOP_K = 8       # experts per token
 I = 704         # moe_intermediate_size; gate_up has 2*I rows
 BLOCK = 16      # elements per E4M3 block scale
+DENSE_I = 2112  # the block's dense MLP intermediate size
 
 __all__ = [
     "H", "E", "TOP_K", "I", "BLOCK", "Router", "Experts",
     "bf16_bits", "make_x", "make_router", "make_expert", "make_experts",
     "make_quant_expert", "make_quant_weights",
-    "zipf_bias", "layer_seed_plan",
+    "zipf_bias", "layer_seed_plan", "DENSE_I", "Block", "make_block",
 ]
 
 
@@ -177,3 +178,31 @@ def make_quant_weights(seed: int, e: int, n: int, k: int, outlier_frac: float = 
 def layer_seed_plan(n_layers: int = 30, base: int = 100) -> list[int]:
     """Seeds of an independently seeded layer stack (layer l uses base + l)."""
     return [base + l for l in range(n_layers)]
+
+
+@dataclasses.dataclass
+class Block:
+    """The full MoE block's parameters besides the experts and the router
+    (bf16 bit patterns): the dense GELU-gated MLP and the five norm weights,
+    and the layer scalar."""
+    dense_gate: np.ndarray      # [Id, H]
+    dense_up: np.ndarray        # [Id, H]
+    dense_down: np.ndarray      # [H, Id]
+    pre_ff_norm: np.ndarray     # [H]
+    post_ff_norm_1: np.ndarray  # [H]
+    pre_ff_norm_2: np.ndarray   # [H]
+    post_ff_norm_2: np.ndarray  # [H]
+    post_ff_norm: np.ndarray    # [H]
+    layer_scalar: np.ndarray    # [1]
+
+
+def make_block(seed: int, h: int = H, di: int = DENSE_I) -> Block:
+    """Dense MLP weights ~ N(0, 0.02); norm weights ~ 1 + N(0, 0.05);
+    layer scalar ~ U(0.5, 1.0); all bf16."""
+    rng = np.random.default_rng(seed)
+    g = rng.standard_normal((di, h), dtype=np.float32) * np.float32(0.02)
+    u = rng.standard_normal((di, h), dtype=np.float32) * np.float32(0.02)
+    d = rng.standard_normal((h, di), dtype=np.float32) * np.float32(0.02)
+    norms = [np.float32(1.0) + rng.standard_normal(h, dtype=np.float32) * np.float32(0.05) for _ in range(5)]
+    ls = np.array([rng.uniform(0.5, 1.0)], np.float32)
+    return Block(bf16_bits(g), bf16_bits(u), bf16_bits(d), *[bf16_bits(n) for n in norms], bf16_bits(ls))

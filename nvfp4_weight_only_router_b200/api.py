@@ -6,6 +6,7 @@ from __future__ import annotations
 import ctypes
 import dataclasses
 
+import numpy as np
 import torch
 
 from . import capi
@@ -174,10 +175,84 @@ class MoeLayer:
         y = torch.empty_like(x)
         return self.forward_into(x, y, stream)
 
+    def forward_dense_into(self, x: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+        """The dense over-read (every token through all 128 experts, weighted
+        by its routing weights): the same y, for measuring the gather's
+        advantage.  Uses its own workspace, sized on first use."""
+        T = x.shape[0]
+        nbytes = capi.moe_forward_dense_workspace_bytes(T, ctypes.byref(self._xs), ctypes.byref(self._rs))
+        if nbytes == 0:
+            raise ValueError(f"T={T} is outside the dense variant's range")
+        if getattr(self, "_dense_ws", None) is None or self._dense_ws.numel() < nbytes:
+            self._dense_ws = _workspace(nbytes, x.device)
+        check(capi.moe_nvfp4_forward_dense(_ptr(x), T, ctypes.byref(self._xs), ctypes.byref(self._rs),
+                                           _ptr(y), _ptr(self._dense_ws), self._dense_ws.numel(),
+                                           _stream(stream)), "moe_nvfp4_forward_dense")
+        return y
+
     def views(self, T: int) -> dict:
         """Intermediate results of the last forward of T tokens, as torch views
         of the workspace (see moe_forward_views in the header)."""
         return forward_views(self, T)
+
+
+@dataclasses.dataclass
+class DenseParts:
+    """The full block's bf16 tensors besides the experts and the router: the
+    dense GELU-gated MLP, the five norm weights and the layer scalar."""
+    dense_gate: torch.Tensor       # [2112, H]
+    dense_up: torch.Tensor         # [2112, H]
+    dense_down: torch.Tensor       # [H, 2112]
+    pre_ff_norm: torch.Tensor      # [H]
+    post_ff_norm_1: torch.Tensor   # [H]
+    pre_ff_norm_2: torch.Tensor    # [H]
+    post_ff_norm_2: torch.Tensor   # [H]
+    post_ff_norm: torch.Tensor     # [H]
+    layer_scalar: torch.Tensor     # [1]
+
+    @staticmethod
+    def from_host(b, device="cuda") -> "DenseParts":
+        """From host bf16 bit patterns (numpy uint16 arrays)."""
+        def bf(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view("int16")).view(torch.bfloat16).to(device)
+        return DenseParts(*(bf(getattr(b, f.name)) for f in dataclasses.fields(DenseParts)))
+
+
+class MoeBlock:
+    """The full feed-forward block of a Gemma-4-26B-A4B layer (dense MLP in
+    parallel with the NVFP4 sparse branch, norms, residual, layer scalar) with
+    a workspace for up to `max_tokens` tokens."""
+
+    def __init__(self, experts: Experts, router: Router, parts: DenseParts, max_tokens: int, eps: float = 1e-6):
+        self.experts, self.router, self.parts = experts, router, parts
+        self._c = capi.moe_block(experts.c_struct(), router.c_struct(), _ptr(parts.dense_gate),
+                                 _ptr(parts.dense_up), _ptr(parts.dense_down), _ptr(parts.pre_ff_norm),
+                                 _ptr(parts.post_ff_norm_1), _ptr(parts.pre_ff_norm_2),
+                                 _ptr(parts.post_ff_norm_2), _ptr(parts.post_ff_norm), _ptr(parts.layer_scalar),
+                                 parts.dense_gate.shape[0], eps)
+        self.max_tokens = int(max_tokens)
+        nbytes = capi.moe_block_workspace_bytes(self.max_tokens, ctypes.byref(self._c))
+        if nbytes == 0:
+            raise ValueError("unsupported block configuration")
+        self.workspace = _workspace(nbytes, experts.gate_up_q.device)
+
+    def forward_into(self, x: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"T={T} exceeds max_tokens={self.max_tokens}")
+        check(capi.moe_block_forward(_ptr(x), T, ctypes.byref(self._c), _ptr(y), _ptr(self.workspace),
+                                     self.workspace.numel(), _stream(stream)), "moe_block_forward")
+        return y
+
+    def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        return self.forward_into(x, torch.empty_like(x), stream)
+
+    def ids(self, T: int) -> torch.Tensor:
+        """The routed ids of the last forward of T tokens."""
+        v = capi.moe_forward_views()
+        check(capi.moe_forward_workspace_views(T, ctypes.byref(self._c.experts), ctypes.byref(self._c.router),
+                                               ctypes.byref(v)), "moe_forward_workspace_views")
+        return self.workspace[v.ids:v.ids + T * TOP_K * 4].view(torch.int32).view(T, TOP_K)
 
 
 def forward_views(layer: MoeLayer, T: int) -> dict:

@@ -53,8 +53,16 @@ class moe_forward_views(ctypes.Structure):
                 ("xexp", c_size_t), ("h", c_size_t)]
 
 
+class moe_block(ctypes.Structure):
+    _fields_ = [("experts", moe_experts), ("router", moe_router), ("dense_gate", c_void_p),
+                ("dense_up", c_void_p), ("dense_down", c_void_p), ("pre_ff_norm", c_void_p),
+                ("post_ff_norm_1", c_void_p), ("pre_ff_norm_2", c_void_p), ("post_ff_norm_2", c_void_p),
+                ("post_ff_norm", c_void_p), ("layer_scalar", c_void_p), ("dense_I", c_int32), ("eps", c_float)]
+
+
 _R = ctypes.POINTER(moe_router)
 _X = ctypes.POINTER(moe_experts)
+_B = ctypes.POINTER(moe_block)
 
 # name -> (restype, argtypes), in the order of the header
 SIGNATURES = {
@@ -69,9 +77,13 @@ SIGNATURES = {
     "moe_route": (c_int32, [c_void_p, c_int32, _R, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_forward_workspace_bytes": (c_size_t, [c_int32, _X, _R]),
     "moe_nvfp4_forward": (c_int32, [c_void_p, c_int32, _X, _R, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_forward_dense_workspace_bytes": (c_size_t, [c_int32, _X, _R]),
+    "moe_nvfp4_forward_dense": (c_int32, [c_void_p, c_int32, _X, _R, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_nvfp4_forward_profiled": (c_int32, [c_void_p, c_int32, _X, _R, c_void_p, c_void_p, c_size_t,
                                              c_void_p, ctypes.POINTER(c_void_p)]),
     "moe_forward_workspace_views": (c_int32, [c_int32, _X, _R, ctypes.POINTER(moe_forward_views)]),
+    "moe_block_workspace_bytes": (c_size_t, [c_int32, _B]),
+    "moe_block_forward": (c_int32, [c_void_p, c_int32, _B, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_permute_workspace_bytes": (c_size_t, [c_int32]),
     "moe_permute": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                               c_void_p]),

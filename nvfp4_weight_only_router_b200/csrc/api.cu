@@ -1,5 +1,6 @@
 // C ABI of the NVFP4 MoE library: argument validation, workspace layout and
 // launch sequencing on the caller's stream.  See include/nvfp4moe.h.
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 
@@ -59,23 +60,28 @@ constexpr int kFusedPermuteMaxSlots = 1024;  // the router's last CTA groups the
 // Largest token count that takes the streaming GEMV path; above it the
 // tensor-core grouped GEMMs run.
 constexpr int kStreamMaxTokens = 256;
+// Largest token count of the dense over-read variant (128 slots per token).
+constexpr int kDenseMaxTokens = 256;
 
 struct FwdLayout {
   Region meta;
-  Region ids, wts, chunk_count, sorted, pos, xexp, xs, h, obuf;
-  int S = 0, nchunks = 0;
+  Region ids, wts, wdense, chunk_count, sorted, pos, xexp, xs, h, obuf;
+  int S = 0, nchunks = 0, spt = kTopK;
   size_t total = 0;
 };
 
-FwdLayout fwd_layout(int T) {
+// dense: the over-read variant (every token through all 128 experts)
+FwdLayout fwd_layout(int T, bool dense = false) {
   FwdLayout L;
   Alloc al;
-  L.S = T * kTopK;
+  L.spt = dense ? kE : kTopK;
+  L.S = T * L.spt;
   L.nchunks = (L.S + 1023) / 1024;
   // zeroed on entry: meta (includes the router's arrival counter)
   L.meta = al.take(sizeof(int) * kMetaInts);
-  L.ids = al.take(sizeof(int) * L.S);
-  L.wts = al.take(sizeof(float) * L.S);
+  L.ids = al.take(sizeof(int) * T * kTopK);
+  L.wts = al.take(sizeof(float) * T * kTopK);
+  if (dense) L.wdense = al.take(sizeof(float) * L.S);
   L.chunk_count = al.take(sizeof(int) * (size_t)L.nchunks * kE);
   L.sorted = al.take(sizeof(int) * L.S);
   L.pos = al.take(sizeof(int) * L.S);
@@ -308,15 +314,19 @@ nvfp4_status moe_forward_workspace_views(int32_t T, const moe_experts* ex, const
   return NVFP4_OK;
 }
 
+// The routed forward.  x_route (null: x) is the router's input, x the
+// experts'; with finalize false the per-slot rows are left in the workspace
+// (for the full block's final kernel) and y is not written.
 static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex,
                                  const moe_router* r, void* y, void* ws, size_t ws_bytes,
-                                 void* stream, void* const* ev) {
-  if (T < 1 || T > 65536 || !x || !y) return NVFP4_ERR_INVALID_ARG;
+                                 void* stream, void* const* ev, bool dense = false,
+                                 const void* x_route = nullptr, bool finalize = true) {
+  if (T < 1 || T > (dense ? kDenseMaxTokens : 65536) || !x || (finalize && !y)) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_experts(ex);
   if (st == NVFP4_OK) st = check_router(r, true);
   if (st != NVFP4_OK) return st;
-  if (!aligned(x, 16) || !aligned(y, 16)) return NVFP4_ERR_ALIGNMENT;
-  const FwdLayout L = fwd_layout(T);
+  if (!aligned(x, 16) || (y && !aligned(y, 16)) || (x_route && !aligned(x_route, 16))) return NVFP4_ERR_ALIGNMENT;
+  const FwdLayout L = fwd_layout(T, dense);
   if (!ws || ws_bytes < L.total) return NVFP4_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
   cudaStream_t s = as_stream(stream);
@@ -339,8 +349,8 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
 
   int32_t* ids = at<int32_t>(ws, L.ids);
   float* wts = at<float>(ws, L.wts);
-  RouteArgs ra = make_route_args(x, T, r, ids, wts, status);
-  const bool fused_permute = ra.few_tokens && L.S <= kFusedPermuteMaxSlots;
+  RouteArgs ra = make_route_args(x_route ? x_route : x, T, r, ids, wts, status);
+  const bool fused_permute = !dense && ra.few_tokens && L.S <= kFusedPermuteMaxSlots;
   if (fused_permute) {
     ra.meta = at<int>(ws, L.meta);
     ra.sorted_slot = at<int>(ws, L.sorted);
@@ -357,7 +367,12 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   pa.sorted_slot = at<int>(ws, L.sorted);
   pa.slot_pos = at<int>(ws, L.pos);
   pa.status = status;
-  if (!fused_permute && (e = launch_permute(pa, s)) != cudaSuccess) return cuda_fail(e);
+  if (dense) {
+    e = launch_dense_permute(ids, wts, T, pa.meta, pa.sorted_slot, pa.slot_pos, at<float>(ws, L.wdense), status, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  } else if (!fused_permute && (e = launch_permute(pa, s)) != cudaSuccess) {
+    return cuda_fail(e);
+  }
 
   ExpertArgs xa;
   xa.gu_q = ex->gate_up_q;
@@ -370,13 +385,14 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   xa.meta = pa.meta;
   xa.sorted_slot = pa.sorted_slot;
   xa.slot_pos = pa.slot_pos;
-  xa.wts = wts;
+  xa.wts = dense ? at<float>(ws, L.wdense) : wts;
+  xa.spt = L.spt;
   xa.xexp = at<int>(ws, L.xexp);
   xa.h = at<__half>(ws, L.h);
   xa.obuf = at<float>(ws, L.obuf);
   xa.y = y;
   xa.T = T;
-  xa.max_active = L.S < kE ? L.S : kE;
+  xa.max_active = L.S < kE ? L.S : kE;  // (the kernels read the active count from meta)
   xa.status = status;
   xa.xs = at<__half>(ws, L.xs);
   // the activations follow their slots into expert order (f16 for the MMAs)
@@ -397,13 +413,139 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
     e = launch_moe_down(xa, nt, s);
     if (e != cudaSuccess || !mark(4)) return cuda_fail(e);
   }
-  if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return cuda_fail(e);
+  if (finalize && ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5))) return cuda_fail(e);
   return NVFP4_OK;
+}
+
+// ------------------------------------------------------------- full block
+namespace {
+
+constexpr int kBlockMaxTokens = 8192;
+constexpr int kMaxSms = 148;  // the workspace holds the dense K splits for up to this many SMs
+
+struct BlockLayout {
+  FwdLayout moe;
+  Region x1, x2, gu_part, hd_hi, hd_lo, dn_part;
+  int sp_gu = 1, sp_dn = 1;
+  size_t total = 0;
+};
+
+BlockLayout block_layout(int T) {
+  BlockLayout L;
+  L.moe = fwd_layout(T);
+  Alloc al;
+  al.cur = L.moe.total;
+  L.sp_gu = dense_splits(0, T, kMaxSms);
+  L.sp_dn = dense_splits(1, T, kMaxSms);
+  L.x1 = al.take(sizeof(uint16_t) * (size_t)T * kH);
+  L.x2 = al.take(sizeof(uint16_t) * (size_t)T * kH);
+  L.gu_part = al.take(sizeof(float) * (size_t)L.sp_gu * T * 2 * kDenseI);
+  L.hd_hi = al.take(sizeof(uint16_t) * (size_t)T * kDenseI);
+  L.hd_lo = al.take(sizeof(uint16_t) * (size_t)T * kDenseI);
+  L.dn_part = al.take(sizeof(float) * (size_t)L.sp_dn * T * kH);
+  L.total = al.cur;
+  return L;
+}
+
+nvfp4_status check_block(const moe_block* b) {
+  if (!b) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_experts(&b->experts);
+  if (st == NVFP4_OK) st = check_router(&b->router, true);
+  if (st != NVFP4_OK) return st;
+  const void* ps[] = {b->dense_gate, b->dense_up, b->dense_down, b->pre_ff_norm, b->post_ff_norm_1,
+                      b->pre_ff_norm_2, b->post_ff_norm_2, b->post_ff_norm, b->layer_scalar};
+  for (const void* q : ps)
+    if (!q) return NVFP4_ERR_INVALID_ARG;
+  if (b->dense_I <= 0 || !(b->eps >= 0.f) || !std::isfinite(b->eps)) return NVFP4_ERR_INVALID_ARG;
+  if (b->dense_I != kDenseI) return NVFP4_ERR_UNSUPPORTED;
+  for (const void* q : ps)
+    if (!aligned(q, 16)) return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+size_t moe_block_workspace_bytes(int32_t T, const moe_block* b) {
+  if (T < 1 || T > kBlockMaxTokens || check_block(b) != NVFP4_OK) return 0;
+  return block_layout(T).total;
+}
+
+nvfp4_status moe_block_forward(const void* x, int32_t T, const moe_block* b, void* y, void* ws, size_t ws_bytes,
+                               void* stream) {
+  if (T < 1 || T > kBlockMaxTokens || !x || !y) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_block(b);
+  if (st != NVFP4_OK) return st;
+  if (!aligned(x, 16) || !aligned(y, 16)) return NVFP4_ERR_ALIGNMENT;
+  const BlockLayout L = block_layout(T);
+  if (!ws || ws_bytes < L.total) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = as_stream(stream);
+  int sms = 0;
+  cudaError_t e = sm_count(&sms);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int sp_gu = std::min(L.sp_gu, dense_splits(0, T, sms));
+  const int sp_dn = std::min(L.sp_dn, dense_splits(1, T, sms));
+  uint16_t* x1 = at<uint16_t>(ws, L.x1);
+  uint16_t* x2 = at<uint16_t>(ws, L.x2);
+  // the two pre-feedforward norms (the MLPs' bf16 inputs)
+  e = launch_block_prenorm(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(b->pre_ff_norm),
+                           static_cast<const uint16_t*>(b->pre_ff_norm_2), b->eps, T, x1, x2, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // the sparse branch: router on the raw residual, experts on x2; per-slot rows stay in ws
+  st = forward_impl(x2, T, &b->experts, &b->router, nullptr, ws, ws_bytes, stream, nullptr, false, x, false);
+  if (st != NVFP4_OK) return st;
+  // the dense branch
+  DenseArgs da;
+  da.w0 = b->dense_gate;
+  da.w1 = b->dense_up;
+  da.b0 = x1;
+  da.b1 = nullptr;
+  da.out = at<float>(ws, L.gu_part);
+  da.T = T;
+  da.splits = sp_gu;
+  da.status = device_status_ptr();
+  if ((e = launch_dense_gate_up(da, s)) != cudaSuccess) return cuda_fail(e);
+  uint16_t* hi = at<uint16_t>(ws, L.hd_hi);
+  uint16_t* lo = at<uint16_t>(ws, L.hd_lo);
+  if ((e = launch_dense_act(da.out, sp_gu, T, hi, lo, s)) != cudaSuccess) return cuda_fail(e);
+  da.w0 = b->dense_down;
+  da.w1 = nullptr;
+  da.b0 = hi;
+  da.b1 = lo;
+  da.out = at<float>(ws, L.dn_part);
+  da.splits = sp_dn;
+  if ((e = launch_dense_down(da, s)) != cudaSuccess) return cuda_fail(e);
+  // the post norms, the residual and the layer scalar
+  BlockFinalArgs fa;
+  fa.x = static_cast<const uint16_t*>(x);
+  fa.obuf = at<float>(ws, L.moe.obuf);
+  fa.slot_pos = at<int>(ws, L.moe.pos);
+  fa.dense = da.out;
+  fa.splits = sp_dn;
+  fa.T = T;
+  fa.post1 = static_cast<const uint16_t*>(b->post_ff_norm_1);
+  fa.post2 = static_cast<const uint16_t*>(b->post_ff_norm_2);
+  fa.post = static_cast<const uint16_t*>(b->post_ff_norm);
+  fa.layer_scalar = static_cast<const uint16_t*>(b->layer_scalar);
+  fa.eps = b->eps;
+  fa.y = y;
+  return cuda_status(launch_block_final(fa, s));
 }
 
 nvfp4_status moe_nvfp4_forward(const void* x, int32_t T, const moe_experts* ex, const moe_router* r,
                                void* y, void* ws, size_t ws_bytes, void* stream) {
   return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, nullptr);
+}
+
+size_t moe_forward_dense_workspace_bytes(int32_t T, const moe_experts* ex, const moe_router* r) {
+  if (T < 1 || T > kDenseMaxTokens || check_experts(ex) != NVFP4_OK || check_router(r, true) != NVFP4_OK)
+    return 0;
+  return fwd_layout(T, true).total;
+}
+
+nvfp4_status moe_nvfp4_forward_dense(const void* x, int32_t T, const moe_experts* ex, const moe_router* r,
+                                     void* y, void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, nullptr, true);
 }
 
 nvfp4_status moe_nvfp4_forward_profiled(const void* x, int32_t T, const moe_experts* ex,

@@ -2,8 +2,9 @@
 // Core AI": the token's output is the router-weighted sum over its top-8
 // experts).  The down GEMMs already multiplied each slot's row by its routing
 // weight and the expert's global scale and stored it at the slot's sorted
-// position; this kernel sums the 8 rows of a token in slot order j = 0..7 and
-// rounds once to bf16, so the result does not depend on launch order.
+// position; this kernel sums the rows of a token in slot order j = 0, 1, ...
+// (8 slots, or 128 in the dense over-read) and rounds once to bf16, so the
+// result does not depend on launch order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -21,9 +22,8 @@ __global__ void __launch_bounds__(256) finalize_kernel(ExpertArgs p) {
   float v[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) v[k] = 0.f;
-#pragma unroll
-  for (int j = 0; j < kTopK; ++j) {
-    const int pos = p.slot_pos[t * kTopK + j];
+  for (int j = 0; j < p.spt; ++j) {
+    const int pos = p.slot_pos[t * p.spt + j];
     if (pos < 0) continue;
     const float4* src = reinterpret_cast<const float4*>(p.obuf + (size_t)pos * kH + c);
     const float4 x0 = __ldcs(src), x1 = __ldcs(src + 1);

@@ -15,6 +15,7 @@ constexpr int kI = 704;           // moe_intermediate_size
 constexpr int kE = 128;           // routed experts
 constexpr int kTopK = 8;          // experts per token
 constexpr int kBlock = 16;        // elements per E4M3 block scale
+constexpr int kDenseI = 2112;     // the full block's dense MLP intermediate_size
 
 // Packed row geometry.
 constexpr int kGuRowBytes = kH / 2;        // 1408: one gate_up row, two codes per byte

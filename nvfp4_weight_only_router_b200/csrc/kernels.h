@@ -64,6 +64,12 @@ struct PermuteArgs {
   int* status;
 };
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
+// The dense over-read's permutation: every token t to every expert e, slot
+// t*128 + e at sorted position e*T + t, with weight w_tj if e = ids[t, j] for
+// some j and 0 otherwise.  meta gets counts T, offsets e*T and all experts
+// active.
+cudaError_t launch_dense_permute(const int32_t* ids, const float* wts, int T, int* meta, int* sorted_slot,
+                                 int* slot_pos, float* wdense, int* status, cudaStream_t st);
 
 struct ExpertArgs {
   const uint8_t* gu_q;
@@ -85,6 +91,7 @@ struct ExpertArgs {
   float* obuf;              // [S, H] per-slot weighted outputs, sorted order
   void* y;                  // bf16 [T, H]
   int T, max_active;
+  int spt;                  // slots per token: 8 (top-8), or 128 (the dense over-read, every expert)
   int* status;
 };
 // y[t] = bf16(sum over the token's 8 slots of obuf, in slot order)
@@ -97,6 +104,47 @@ cudaError_t launch_down_stream(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_moe_gate_up(const ExpertArgs& a, int nt, cudaStream_t st);
 cudaError_t launch_moe_down(const ExpertArgs& a, int nt, cudaStream_t st);
+
+// The full block's dense MLP GEMMs (bf16 x bf16 -> fp32 on tcgen05).
+//   gate_up: w0 = gate [2112, H], w1 = up [2112, H], b0 = X [T, H] (bf16);
+//            out [splits][T][2 * 2112]: gate rows 0..2111, then up rows
+//   down:    w0 = down [H, 2112], b0 / b1 = the gated hidden's bf16 high and
+//            low parts [T, 2112]; out [splits][T][H]
+// Each K split writes its own slab of out (the consumer sums them in order).
+struct DenseArgs {
+  const void* w0;
+  const void* w1;
+  const void* b0;
+  const void* b1;
+  float* out;
+  int T;
+  int splits;               // K splits (dense_splits for this T, or fewer)
+  int* status;
+};
+cudaError_t launch_dense_gate_up(const DenseArgs& a, cudaStream_t st);
+cudaError_t launch_dense_down(const DenseArgs& a, cudaStream_t st);
+// K splits that give every one of `sms` SMs a tile for T tokens (mode 0
+// gate_up, 1 down); 1 when the row and token tiles already do.
+int dense_splits(int mode, int T, int sms);
+
+// The full block's per-token kernels.
+cudaError_t launch_block_prenorm(const uint16_t* x, const uint16_t* g1, const uint16_t* g2, float eps, int T,
+                                 uint16_t* x1, uint16_t* x2, cudaStream_t st);
+cudaError_t launch_dense_act(const float* part, int splits, int T, uint16_t* hi, uint16_t* lo, cudaStream_t st);
+struct BlockFinalArgs {
+  const uint16_t* x;        // bf16 [T, H] the residual
+  const float* obuf;        // [S, H] per-slot rows of the sparse branch (x w x G_d)
+  const int* slot_pos;      // [T*8]
+  const float* dense;       // [splits, T, H] dense-branch partials
+  int splits, T;
+  const uint16_t* post1;    // post_feedforward_layernorm_1 weight
+  const uint16_t* post2;    // post_feedforward_layernorm_2 weight
+  const uint16_t* post;     // post_feedforward_layernorm weight
+  const uint16_t* layer_scalar;
+  float eps;
+  void* y;                  // bf16 [T, H]
+};
+cudaError_t launch_block_final(const BlockFinalArgs& a, cudaStream_t st);
 
 // 2-D TMA tensor map: `inner` elements per row, `outer` rows, `pitch` bytes
 // between rows, box of box_inner x box_outer; false if the driver refuses it.

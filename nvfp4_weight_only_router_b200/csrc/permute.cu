@@ -159,7 +159,48 @@ __global__ void __launch_bounds__(kChunk) permute_scatter_kernel(PermuteArgs a) 
   }
 }
 
+// One thread per dense slot s = t*128 + e: its sorted position e*T + t, and
+// its weight (the token's routing weight for e, 0 if e is not among its
+// ids).  Block 0 also writes the meta block.
+__global__ void __launch_bounds__(256) dense_permute_kernel(const int32_t* __restrict__ ids,
+                                                            const float* __restrict__ wts, int T,
+                                                            int* __restrict__ meta, int* __restrict__ sorted_slot,
+                                                            int* __restrict__ slot_pos, float* __restrict__ wdense,
+                                                            int* status) {
+  const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (blockIdx.x == 0 && threadIdx.x <= kE) {
+    const int e = threadIdx.x;
+    if (e < kE) {
+      meta[kMetaCounts + e] = T;
+      meta[kMetaAct + e] = e;
+    }
+    meta[kMetaOffsets + e] = e * T;
+    if (e == 0) meta[kMetaNAct] = kE;
+  }
+  if (s >= (int64_t)T * kE) return;
+  const int t = (int)(s / kE), e = (int)(s % kE);
+  float w = 0.f;
+#pragma unroll
+  for (int j = 0; j < kTopK; ++j) {
+    const int id = ids[t * kTopK + j];
+    if (id < 0 || id >= kE) record_status(status, kStatusDevice);
+    if (id == e) w = wts[t * kTopK + j];
+  }
+  const int pos = e * T + t;
+  sorted_slot[pos] = (int)s;
+  slot_pos[s] = pos;
+  wdense[s] = w;
+}
+
 }  // namespace
+
+cudaError_t launch_dense_permute(const int32_t* ids, const float* wts, int T, int* meta, int* sorted_slot,
+                                 int* slot_pos, float* wdense, int* status, cudaStream_t st) {
+  const int64_t n = (int64_t)T * kE;
+  dense_permute_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(ids, wts, T, meta, sorted_slot, slot_pos, wdense,
+                                                                      status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
   permute_count_kernel<<<a.nchunks, kChunk, 0, st>>>(a);

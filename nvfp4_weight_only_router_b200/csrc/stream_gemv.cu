@@ -473,7 +473,7 @@ cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t st) {
   // (row, block) with the 128B swizzle
   CUtensorMap tm_x8, tm_x16;
   {
-    const uint64_t S = (uint64_t)a.T * kTopK;
+    const uint64_t S = (uint64_t)a.T * a.spt;
     const int KX = C::KX;
     const uint64_t dims[3] = {64, (uint64_t)(KX / 64), S};
     const uint64_t pitch[2] = {128, (uint64_t)KX * 2};

@@ -497,7 +497,7 @@ cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
   const int smem = (int)sizeof(MoeSmem<KIND, NT>) + 1024;  // + alignment slack
   cudaError_t err = configure_kernel_once((const void*)tc_moe_kernel<KIND, NT>, smem);
   if (err != cudaSuccess) return err;
-  const uint64_t S = (uint64_t)a.T * kTopK;
+  const uint64_t S = (uint64_t)a.T * a.spt;
   CUtensorMap tm_x, tm_w;
   bool ok;
   if (KIND == kGateUp) {
@@ -527,7 +527,7 @@ cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
 // stores.
 __global__ void __launch_bounds__(256) gather_sorted_kernel(const uint16_t* __restrict__ x,
                                                             const int* __restrict__ sorted_slot,
-                                                            const int* __restrict__ meta, int T,
+                                                            const int* __restrict__ meta, int T, int spt,
                                                             __half* __restrict__ xs, int* __restrict__ xexp,
                                                             int* status) {
   constexpr int per_row = kH / 8;              // 352
@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(256) gather_sorted_kernel(const uint16_t* __re
   const int S = meta[kMetaOffsets + kE];
   const int lane = threadIdx.x & 31;
   for (int pos = blockIdx.x * 8 + (threadIdx.x >> 5); pos < S; pos += gridDim.x * 8) {
-    int tok = sorted_slot[pos] / kTopK;
+    int tok = sorted_slot[pos] / spt;
     if (tok < 0 || tok >= T) {
       record_status(status, kStatusDevice);
       tok = 0;
@@ -577,10 +577,10 @@ __global__ void __launch_bounds__(256) gather_sorted_kernel(const uint16_t* __re
 }  // namespace
 
 cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st) {
-  const int64_t rows = (int64_t)a.T * kTopK;
+  const int64_t rows = (int64_t)a.T * a.spt;
   int blocks = (int)((rows + 7) / 8);
   if (blocks > 148 * 32) blocks = 148 * 32;
-  gather_sorted_kernel<<<blocks, 256, 0, st>>>(a.x, a.sorted_slot, a.meta, a.T, a.xs, a.xexp, a.status);
+  gather_sorted_kernel<<<blocks, 256, 0, st>>>(a.x, a.sorted_slot, a.meta, a.T, a.spt, a.xs, a.xexp, a.status);
   return cudaGetLastError();
 }
 

@@ -23,10 +23,14 @@ Sources (page title, section):
     to 128, fp32 softmax, top-8, renormalise, x per_expert_scale; GELU-tanh
     gated experts).
 
+  * The same card's layer dataflow listing, for the full block (oracle/block):
+    a dense GELU-gated MLP (intermediate 2112) in parallel with the sparse
+    branch, five norms, the router on the raw residual, and layer_scalar.
+
 Parity pins: every function here is pinned by a `-m "not gpu"` test against
 closed forms, library routines (torch float8_e4m3fn, torch softmax/gelu/rms_norm,
 numpy matmul), exhaustive enumeration or brute force on tiny inputs.  The
 pages' own verification numbers need trained weights that are not available,
 so the forward pass is pinned by invariants and brute force only.
 """
-from . import formats, quantize, moe  # noqa: F401
+from . import formats, quantize, moe, block  # noqa: F401

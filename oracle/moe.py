@@ -127,16 +127,18 @@ def expert_hidden(xe: np.ndarray, wgu: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------- forward (a6)
-def forward(x_bits, experts, router, ids_override=None, return_parts=False):
+def forward(x_bits, experts, router, ids_override=None, return_parts=False, route_bits=None):
     """The MoE branch y = sum_j w_j * expert_{ids_j}(x), float64.
 
-    Both the router and the experts read the same x (the pre- and
-    post-feedforward norms of the full block are outside this branch).
+    By default the router and the experts read the same x (the branch on its
+    own).  In the full block the router reads the raw residual while the
+    experts read its pre-feedforward norm (the layer dataflow listing):
+    `route_bits` is then the router's input and `x_bits` the experts'.
     Returns y64 [T, H] (float64) or, with return_parts, a dict that also holds
     ids, weights, logits and the bf16-rounded output."""
     x = bf16_to_f64(x_bits)
     T, H = x.shape
-    ids, w, logits = route(x_bits, router, ids_override)
+    ids, w, logits = route(x_bits if route_bits is None else route_bits, router, ids_override)
     counts, offsets, sorted_slot, _ = permute(ids, experts.E)
     k = ids.shape[1]
     y = np.zeros((T, H), np.float64)

@@ -25,7 +25,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported(capi):
     names = header_functions()
-    assert len(names) == 18
+    assert len(names) == 22
     for n in names:
         assert hasattr(capi.lib, n), n
         assert n in capi.SIGNATURES, n
@@ -162,3 +162,41 @@ def test_last_cuda_error_after_a_failed_call_without_a_device(capi):
     P = 4096
     assert capi.nvfp4_quantize_noalloc(P, 1, 16, 32, P, P, P, None) == capi.NVFP4_ERR_CUDA
     assert capi.lib.nvfp4_last_cuda_error().decode() != "no error"
+
+
+def test_dense_variant_validation(capi):
+    c = capi
+    r, x = _router(c), _experts(c)
+    assert c.moe_forward_dense_workspace_bytes(0, ctypes.byref(x), ctypes.byref(r)) == 0
+    assert c.moe_forward_dense_workspace_bytes(257, ctypes.byref(x), ctypes.byref(r)) == 0
+    small = c.moe_forward_dense_workspace_bytes(1, ctypes.byref(x), ctypes.byref(r))
+    # 128 slots per token instead of 8: far more workspace than the routed forward
+    assert small > 8 * c.moe_forward_workspace_bytes(1, ctypes.byref(x), ctypes.byref(r))
+    P = 4096
+    assert c.moe_nvfp4_forward_dense(P, 257, ctypes.byref(x), ctypes.byref(r), P, P, small, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_nvfp4_forward_dense(P, 1, ctypes.byref(x), ctypes.byref(r), P, P, small - 1, None) == c.NVFP4_ERR_WORKSPACE
+
+
+def _block(c, dense_I=2112, ptr=4096, eps=1e-6):
+    P = ptr
+    return c.moe_block(_experts(c), _router(c), P, P, P, P, P, P, P, P, P, dense_I, eps)
+
+
+def test_block_validation(capi):
+    c = capi
+    b = _block(c)
+    sizes = [c.moe_block_workspace_bytes(T, ctypes.byref(b)) for T in (1, 64, 4096)]
+    assert 0 < sizes[0] < sizes[1] < sizes[2]
+    assert c.moe_block_workspace_bytes(8193, ctypes.byref(b)) == 0
+    assert c.moe_block_workspace_bytes(1, ctypes.byref(_block(c, dense_I=2048))) == 0
+    P = 4096
+    ws = sizes[0]
+    assert c.moe_block_forward(P, 1, ctypes.byref(b), P, P, ws - 1, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.moe_block_forward(None, 1, ctypes.byref(b), P, P, ws, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_block_forward(P, 1, ctypes.byref(_block(c, dense_I=2048)), P, P, ws, None) == c.NVFP4_ERR_UNSUPPORTED
+    assert c.moe_block_forward(P, 1, ctypes.byref(_block(c, eps=-1.0)), P, P, ws, None) == c.NVFP4_ERR_INVALID_ARG
+    bad = _block(c)
+    bad.post_ff_norm = 4096 + 8
+    assert c.moe_block_forward(P, 1, ctypes.byref(bad), P, P, ws, None) == c.NVFP4_ERR_ALIGNMENT
+    bad.post_ff_norm = None
+    assert c.moe_block_forward(P, 1, ctypes.byref(bad), P, P, ws, None) == c.NVFP4_ERR_INVALID_ARG

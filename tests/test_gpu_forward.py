@@ -276,3 +276,25 @@ def test_stack_chained_layers(dev):
     d_gpu = res.double().cpu().numpy() - F.bf16_to_f64(x0)
     d_o = res_o - F.bf16_to_f64(x0)
     assert np.linalg.norm(d_gpu - d_o) / np.linalg.norm(d_o) <= 2e-3
+
+
+# ------------------------------------------------------ dense over-read
+@pytest.mark.parametrize("T", [1, 8, 33])
+def test_forward_dense_over_read(layer0, dev, T):
+    """The dense over-read (every token through all 128 experts, weighted by
+    its routing weights, 0 for unselected experts) computes the same branch:
+    its y meets the forward bar against the oracle, like the routed forward's."""
+    ex, rt = layer0["ex"], layer0["rt"]
+    layer = lib.MoeLayer(layer0["dex"], layer0["drt"], max_tokens=T)
+    x = gen.make_x(71 + T, T)
+    xd = bf16_to_dev(x, dev)
+    y_sparse = layer(xd)
+    ids = layer.views(T)["ids"].cpu().numpy()
+    y_dense = layer.forward_dense_into(xd, torch.empty_like(xd))
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0
+    ids0, _, logits = M.route(x, rt)
+    differ = check_ids(ids, ids0, logits)
+    y64 = _oracle_y(x, ex, rt, ids, differ)
+    check_forward(bf16_from_dev(y_dense), y64)
+    check_forward(bf16_from_dev(y_sparse), y64)
