@@ -2,8 +2,8 @@
 """Benchmark of the NVFP4 weight-only MoE branch on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode64|decode1|dense1|prefill4096|block64|block4096|
-                                stack30|quantize]
+                    [--workload decode64|decode1|dense1|aff4_64|prefill4096|block64|
+                                block4096|stack30|quantize]
 
 A step is one pass of the whole hot path -- route, permute, gate_up + GELU,
 down, combine -- over one batch of synthetic tokens (the default workload:
@@ -37,6 +37,8 @@ METRIC = "MoE-layer tokens/s; decode HBM GB/s vs ~8 TB/s; prefill TFLOP/s vs bf1
 GU_EXPERT_BYTES = 1408 * 1408 + 1408 * 176 + 4        # packed + scales + global
 DN_EXPERT_BYTES = 2816 * 352 + 2816 * 44 + 4
 EXPERT_BYTES = GU_EXPERT_BYTES + DN_EXPERT_BYTES        # 3,345,416
+AFF4_GU_BYTES = 1408 * 1408 + 1408 * 88 * 4             # codes + fp16 scales and biases per 32
+AFF4_EXPERT_BYTES = AFF4_GU_BYTES + 2816 * 352 + 2816 * 22 * 4   # 3,717,120
 ROUTER_BYTES = 128 * 2816 * 2 + 2816 * 2 + 128 * 2       # 726,784 (bf16 proj, scale, pes)
 FLUSH_BYTES = 256 << 20
 
@@ -73,6 +75,8 @@ WORKLOADS = {
     "decode1": {"T": 1, "layers": 1, "zipf": False, "desc": "one MoE layer, decode T=1"},
     "prefill4096": {"T": 4096, "layers": 1, "zipf": True,
                     "desc": "one MoE layer, prefill T=4096, Zipf(1.1)-skewed router bias"},
+    "aff4_64": {"T": 64, "layers": 1, "zipf": False, "aff4": True,
+                "desc": "one MoE layer with aff4 experts (u4, fp16 scale+bias per 32), decode T=64"},
     "dense1": {"T": 1, "layers": 1, "zipf": False, "dense": True,
                "desc": "one MoE layer, decode T=1, dense over-read: all 128 experts per token (ablation)"},
     "block64": {"T": 64, "layers": 1, "zipf": False, "block": True,
@@ -170,6 +174,9 @@ class OracleSample:
             self.what = "oracle quantize of 1 of the 128 expert tensors [1408,2816]"
             return
         self.ex = gen.make_experts(0 if wl["layers"] == 1 else 100)
+        if wl.get("aff4"):
+            from oracle import aff4 as A
+            self.ex = A.Aff4Experts(*gen.make_aff4_experts(9))
         self.rt = gen.make_router(1, bias=gen.zipf_bias(7) if wl["zipf"] else None)
         self.x = gen.make_x(10_000, max(wl["T"], tokens))[:tokens]
         self.block = None
@@ -334,6 +341,9 @@ def measure(ctx, workload, args, cpu_baseline=True):
             if wl.get("block"):
                 parts = lib.DenseParts.from_host(gen.make_block(200), dev)
                 layers.append(lib.MoeBlock(ctx.experts(sd), lib.Router.from_host(rt, dev), parts, max_tokens=T))
+            elif wl.get("aff4"):
+                layers.append(lib.Aff4Layer(lib.Aff4Experts.from_host(gen.make_aff4_experts(9), dev),
+                                            lib.Router.from_host(rt, dev), max_tokens=T))
             else:
                 layers.append(lib.MoeLayer(ctx.experts(sd), lib.Router.from_host(rt, dev), max_tokens=T))
         xs_host = np.stack([gen.make_x(replica_x_seed(rank, n_pool, i), T) for i in range(n_pool)])
@@ -349,7 +359,7 @@ def measure(ctx, workload, args, cpu_baseline=True):
             st = torch.cuda.current_stream().cuda_stream
             if wl.get("dense"):
                 layer.forward_dense_into(xin, yout)
-            elif wl.get("block"):
+            elif wl.get("block") or wl.get("aff4"):
                 layer.forward_into(xin, yout)
             elif profiled:
                 arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
@@ -435,9 +445,9 @@ def measure(ctx, workload, args, cpu_baseline=True):
         end.record()
         torch.cuda.synchronize()
         step_ms.append(start.elapsed_time(end))
-        if workload != "quantize" and not wl.get("block"):
+        if workload != "quantize" and not (wl.get("block") or wl.get("aff4")):
             act_counts.append(int((layers[0].views(T)["counts"] > 0).sum().item()))
-        elif wl.get("block"):
+        elif wl.get("block") or wl.get("aff4"):
             act_counts.append(int(torch.unique(layers[0].ids(T)).numel()))
     torch.cuda.synchronize()
     # phase breakdown (and the dominant kernel's duration for the roofline):
@@ -446,7 +456,7 @@ def measure(ctx, workload, args, cpu_baseline=True):
     prof_ms = []
     if workload != "quantize":
         for k in range(args.steps):
-            if wl.get("dense") or wl.get("block"):
+            if wl.get("dense") or wl.get("block") or wl.get("aff4"):
                 break  # these variants record no phase events
             ctx.flush.zero_()
             prepare(k)
@@ -542,6 +552,12 @@ def measure(ctx, workload, args, cpu_baseline=True):
             roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM + GELU (tcgen05)", "achieved": ach,
                     "peak": ctx.tc_peak, "unit": "TFLOP/s", "traffic": traffic,
                     "peak_kind": ctx.peak_kind + " burst bf16", "algorithmic_per_launch": gu_flops}
+        elif wl.get("aff4"):
+            nbytes = (n_act * AFF4_EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2).mean()
+            ach = nbytes / (ms_per_step / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": "whole aff4 step (no phase split)", "achieved": ach,
+                    "peak": ctx.hbm_peak, "unit": "GB/s", "traffic": traffic, "peak_kind": ctx.peak_kind,
+                    "algorithmic_per_launch": float(nbytes)}
         elif wl.get("dense"):
             # no phase split: the whole step's algorithmic bytes (all 128 experts)
             ach = (n_act * EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2).mean() / (ms_per_step / 1e3) / 1e9
@@ -557,7 +573,7 @@ def measure(ctx, workload, args, cpu_baseline=True):
         roof["frac"] = roof["achieved"] / roof["peak"]
         step_bytes = n_act * EXPERT_BYTES + ROUTER_BYTES + 2 * T * 2816 * 2
         extra = {
-            "phase_ms_mean": None if (wl.get("dense") or wl.get("block")) else dict(zip(["route", "permute", "gate_up", "down", "combine"],
+            "phase_ms_mean": None if (wl.get("dense") or wl.get("block") or wl.get("aff4")) else dict(zip(["route", "permute", "gate_up", "down", "combine"],
                                                                  [float(v) for v in ph.mean(0)])),
             "ms_per_step_with_phase_events": float(np.mean(prof_ms)) if prof_ms else None,
             "active_experts_mean": float(n_act.mean()),

@@ -208,6 +208,37 @@ NVFP4MOE_API nvfp4_status moe_nvfp4_forward(const void* x_dev, int32_t T, const 
                                const moe_router* router, void* y_dev,
                                void* ws_dev, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_aff4_forward: moe_nvfp4_forward with the experts in the aff4 codec
+ * ("Gemma 4 26B-A4B (MoE) - Core AI", "Compression recipe": affine int4 with
+ * an fp16 scale and bias per (output row, K-block of 32); a q4_0 grid
+ * w = (q - 8) d is the block with scale = d, bias = -8 d):
+ *   w = q * scale + bias,  q the unsigned 4-bit code.
+ * The same router, permutation, grouped kernels, combine and output; each
+ * weight is formed in f16 by one fma (rounded once) before the MMA.
+ *   gate_up_q u8 [E, 2I, H/2]  (rows 0..I-1 gate, I..2I-1 up; element 2j in
+ *             the low nibble of byte j)
+ *   gate_up_s, gate_up_b fp16 [E, 2I, H/32]
+ *   down_q u8 [E, H, I/2];  down_s, down_b fp16 [E, H, I/32]
+ * Same requirements and workspace size as moe_nvfp4_forward
+ * (moe_aff4_forward_workspace_bytes). */
+typedef struct {
+  const uint8_t* gate_up_q;
+  const void* gate_up_s;   /* fp16 */
+  const void* gate_up_b;   /* fp16 */
+  const uint8_t* down_q;
+  const void* down_s;      /* fp16 */
+  const void* down_b;      /* fp16 */
+  int32_t E;               /* must be 128 */
+  int32_t H;               /* must be 2816 */
+  int32_t I;               /* must be 704 */
+} moe_experts_aff4;
+NVFP4MOE_API size_t moe_aff4_forward_workspace_bytes(int32_t T, const moe_experts_aff4* experts,
+                                                     const moe_router* router);
+NVFP4MOE_API nvfp4_status moe_aff4_forward(const void* x_dev, int32_t T, const moe_experts_aff4* experts,
+                                           const moe_router* router, void* y_dev, void* ws_dev, size_t ws_bytes,
+                                           void* stream);
+
 /* moe_nvfp4_forward_dense: the same output as moe_nvfp4_forward computed the
  * way a runtime without a gather kernel does it ("Gemma 4 26B-A4B (MoE) -
  * Core AI", "Compression recipe": without the gather kernel the sparse

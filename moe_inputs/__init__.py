@@ -30,7 +30,7 @@ __all__ = [
     "H", "E", "TOP_K", "I", "BLOCK", "Router", "Experts",
     "bf16_bits", "make_x", "make_router", "make_expert", "make_experts",
     "make_quant_expert", "make_quant_weights",
-    "zipf_bias", "layer_seed_plan", "DENSE_I", "Block", "make_block",
+    "zipf_bias", "layer_seed_plan", "DENSE_I", "Block", "make_block", "make_aff4_experts",
 ]
 
 
@@ -206,3 +206,30 @@ def make_block(seed: int, h: int = H, di: int = DENSE_I) -> Block:
     norms = [np.float32(1.0) + rng.standard_normal(h, dtype=np.float32) * np.float32(0.05) for _ in range(5)]
     ls = np.array([rng.uniform(0.5, 1.0)], np.float32)
     return Block(bf16_bits(g), bf16_bits(u), bf16_bits(d), *[bf16_bits(n) for n in norms], bf16_bits(ls))
+
+
+def make_aff4_experts(seed: int, e: int = E, h: int = H, i: int = I):
+    """A layer's experts in the aff4 codec, generated directly in packed form
+    (no quantiser): uniformly random 4-bit codes; per (row, K-block of 32) an
+    fp16 scale ~ U(2e-4, 8e-4) and an fp16 bias = -scale * U(6, 9) (a grid
+    centred near zero, as the q4_0 form w = (q - 8) d gives).  Expert j is
+    drawn from default_rng([seed, 1000 + j]).  Returns oracle-shaped arrays:
+    (gate_up_q, gate_up_s, gate_up_b, down_q, down_s, down_b) with the scales
+    and biases as fp16 bit patterns."""
+    def f16(a):
+        return np.asarray(a, np.float32).astype(np.float16).view(np.uint16)
+    gq = np.empty((e, 2 * i, h // 2), np.uint8)
+    gs = np.empty((e, 2 * i, h // 32), np.uint16)
+    gb = np.empty_like(gs)
+    dq = np.empty((e, h, i // 2), np.uint8)
+    ds = np.empty((e, h, i // 32), np.uint16)
+    db = np.empty_like(ds)
+    for j in range(e):
+        rng = np.random.default_rng([seed, 1000 + j])
+        gq[j] = np.frombuffer(rng.bytes(2 * i * h // 2), np.uint8).reshape(2 * i, h // 2)
+        s = rng.uniform(2e-4, 8e-4, size=(2 * i, h // 32)).astype(np.float32)
+        gs[j], gb[j] = f16(s), f16(-s * rng.uniform(6, 9, size=s.shape).astype(np.float32))
+        dq[j] = np.frombuffer(rng.bytes(h * i // 2), np.uint8).reshape(h, i // 2)
+        s = rng.uniform(2e-4, 8e-4, size=(h, i // 32)).astype(np.float32)
+        ds[j], db[j] = f16(s), f16(-s * rng.uniform(6, 9, size=s.shape).astype(np.float32))
+    return gq, gs, gb, dq, ds, db

@@ -197,6 +197,75 @@ class MoeLayer:
 
 
 @dataclasses.dataclass
+class Aff4Experts:
+    """Expert stacks in the aff4 codec on the device: u8 codes, fp16 scales
+    and biases per (row, K-block of 32) (layouts of moe_experts_aff4)."""
+    gate_up_q: torch.Tensor
+    gate_up_s: torch.Tensor
+    gate_up_b: torch.Tensor
+    down_q: torch.Tensor
+    down_s: torch.Tensor
+    down_b: torch.Tensor
+
+    def c_struct(self) -> capi.moe_experts_aff4:
+        return capi.moe_experts_aff4(_ptr(self.gate_up_q), _ptr(self.gate_up_s), _ptr(self.gate_up_b),
+                                     _ptr(self.down_q), _ptr(self.down_s), _ptr(self.down_b),
+                                     self.gate_up_q.shape[0], self.gate_up_q.shape[2] * 2,
+                                     self.down_q.shape[2] * 2)
+
+    @staticmethod
+    def from_host(arrays, device="cuda") -> "Aff4Experts":
+        """From host arrays (gate_up_q, gate_up_s, gate_up_b, down_q, down_s,
+        down_b): u8 codes and fp16 bit patterns (uint16)."""
+        def t(a):
+            a = np.ascontiguousarray(a)
+            if a.dtype == np.uint16:
+                return torch.from_numpy(a.view(np.int16)).view(torch.float16).to(device)
+            return torch.from_numpy(a).to(device)
+        return Aff4Experts(*(t(a) for a in arrays))
+
+
+class Aff4Layer:
+    """One sparse MoE branch with aff4 experts and a workspace for up to
+    `max_tokens` tokens (moe_aff4_forward)."""
+
+    def __init__(self, experts: Aff4Experts, router: Router, max_tokens: int):
+        self.experts, self.router = experts, router
+        self._xs, self._rs = experts.c_struct(), router.c_struct()
+        self.max_tokens = int(max_tokens)
+        nbytes = capi.moe_aff4_forward_workspace_bytes(self.max_tokens, ctypes.byref(self._xs),
+                                                       ctypes.byref(self._rs))
+        if nbytes == 0:
+            raise ValueError("unsupported experts/router configuration")
+        self.workspace = _workspace(nbytes, experts.gate_up_q.device)
+
+    def forward_into(self, x: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"T={T} exceeds max_tokens={self.max_tokens}")
+        check(capi.moe_aff4_forward(_ptr(x), T, ctypes.byref(self._xs), ctypes.byref(self._rs), _ptr(y),
+                                    _ptr(self.workspace), self.workspace.numel(), _stream(stream)),
+              "moe_aff4_forward")
+        return y
+
+    def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        return self.forward_into(x, torch.empty_like(x), stream)
+
+    def ids(self, T: int) -> torch.Tensor:
+        """The routed ids of the last forward of T tokens.  The workspace
+        layout is the NVFP4 forward's (it depends on T only), so the view
+        offsets come from moe_forward_workspace_views with the same pointers
+        standing in for an NVFP4 stack."""
+        e = self._xs
+        stand_in = capi.moe_experts(e.gate_up_q, e.gate_up_s, e.gate_up_s, e.down_q, e.down_s, e.down_s,
+                                    e.E, e.H, e.I)
+        v = capi.moe_forward_views()
+        check(capi.moe_forward_workspace_views(T, ctypes.byref(stand_in), ctypes.byref(self._rs), ctypes.byref(v)),
+              "moe_forward_workspace_views")
+        return self.workspace[v.ids:v.ids + T * TOP_K * 4].view(torch.int32).view(T, TOP_K)
+
+
+@dataclasses.dataclass
 class DenseParts:
     """The full block's bf16 tensors besides the experts and the router: the
     dense GELU-gated MLP, the five norm weights and the layer scalar."""

@@ -53,6 +53,12 @@ class moe_forward_views(ctypes.Structure):
                 ("xexp", c_size_t), ("h", c_size_t)]
 
 
+class moe_experts_aff4(ctypes.Structure):
+    _fields_ = [("gate_up_q", c_void_p), ("gate_up_s", c_void_p), ("gate_up_b", c_void_p),
+                ("down_q", c_void_p), ("down_s", c_void_p), ("down_b", c_void_p),
+                ("E", c_int32), ("H", c_int32), ("I", c_int32)]
+
+
 class moe_block(ctypes.Structure):
     _fields_ = [("experts", moe_experts), ("router", moe_router), ("dense_gate", c_void_p),
                 ("dense_up", c_void_p), ("dense_down", c_void_p), ("pre_ff_norm", c_void_p),
@@ -63,6 +69,7 @@ class moe_block(ctypes.Structure):
 _R = ctypes.POINTER(moe_router)
 _X = ctypes.POINTER(moe_experts)
 _B = ctypes.POINTER(moe_block)
+_A = ctypes.POINTER(moe_experts_aff4)
 
 # name -> (restype, argtypes), in the order of the header
 SIGNATURES = {
@@ -77,6 +84,8 @@ SIGNATURES = {
     "moe_route": (c_int32, [c_void_p, c_int32, _R, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_forward_workspace_bytes": (c_size_t, [c_int32, _X, _R]),
     "moe_nvfp4_forward": (c_int32, [c_void_p, c_int32, _X, _R, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_aff4_forward_workspace_bytes": (c_size_t, [c_int32, _A, _R]),
+    "moe_aff4_forward": (c_int32, [c_void_p, c_int32, _A, _R, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_forward_dense_workspace_bytes": (c_size_t, [c_int32, _X, _R]),
     "moe_nvfp4_forward_dense": (c_int32, [c_void_p, c_int32, _X, _R, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_nvfp4_forward_profiled": (c_int32, [c_void_p, c_int32, _X, _R, c_void_p, c_void_p, c_size_t,

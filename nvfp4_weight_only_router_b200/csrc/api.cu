@@ -154,6 +154,49 @@ nvfp4_status check_experts(const moe_experts* x) {
   return NVFP4_OK;
 }
 
+// The expert stacks of either codec, as the kernels take them.
+struct ExpertPtrs {
+  int codec = kCodecNvfp4;
+  const uint8_t *gu_q = nullptr, *gu_s = nullptr, *dn_q = nullptr, *dn_s = nullptr;
+  const float *gu_g = nullptr, *dn_g = nullptr;
+  const uint16_t *gu_b = nullptr, *dn_b = nullptr;
+};
+
+ExpertPtrs nvfp4_ptrs(const moe_experts* x) {
+  ExpertPtrs e;
+  e.codec = kCodecNvfp4;
+  e.gu_q = x->gate_up_q;
+  e.gu_s = x->gate_up_s;
+  e.gu_g = x->gate_up_g;
+  e.dn_q = x->down_q;
+  e.dn_s = x->down_s;
+  e.dn_g = x->down_g;
+  return e;
+}
+
+nvfp4_status check_experts_aff4(const moe_experts_aff4* x) {
+  if (!x || !x->gate_up_q || !x->gate_up_s || !x->gate_up_b || !x->down_q || !x->down_s || !x->down_b)
+    return NVFP4_ERR_INVALID_ARG;
+  if (x->E <= 0 || x->H <= 0 || x->I <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (x->E != kE || x->H != kH || x->I != kI) return NVFP4_ERR_UNSUPPORTED;
+  const void* ps[] = {x->gate_up_q, x->gate_up_s, x->gate_up_b, x->down_q, x->down_s, x->down_b};
+  for (const void* p : ps)
+    if (!aligned(p, 16)) return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+ExpertPtrs aff4_ptrs(const moe_experts_aff4* x) {
+  ExpertPtrs e;
+  e.codec = kCodecAff4;
+  e.gu_q = x->gate_up_q;
+  e.gu_s = static_cast<const uint8_t*>(x->gate_up_s);
+  e.gu_b = static_cast<const uint16_t*>(x->gate_up_b);
+  e.dn_q = x->down_q;
+  e.dn_s = static_cast<const uint8_t*>(x->down_s);
+  e.dn_b = static_cast<const uint16_t*>(x->down_b);
+  return e;
+}
+
 RouteArgs make_route_args(const void* x, int T, const moe_router* r, int32_t* ids, float* wts, int* status) {
   RouteArgs a;
   a.x = static_cast<const uint16_t*>(x);
@@ -317,13 +360,12 @@ nvfp4_status moe_forward_workspace_views(int32_t T, const moe_experts* ex, const
 // The routed forward.  x_route (null: x) is the router's input, x the
 // experts'; with finalize false the per-slot rows are left in the workspace
 // (for the full block's final kernel) and y is not written.
-static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex,
+static nvfp4_status forward_impl(const void* x, int32_t T, const ExpertPtrs& ex,
                                  const moe_router* r, void* y, void* ws, size_t ws_bytes,
                                  void* stream, void* const* ev, bool dense = false,
                                  const void* x_route = nullptr, bool finalize = true) {
   if (T < 1 || T > (dense ? kDenseMaxTokens : 65536) || !x || (finalize && !y)) return NVFP4_ERR_INVALID_ARG;
-  nvfp4_status st = check_experts(ex);
-  if (st == NVFP4_OK) st = check_router(r, true);
+  nvfp4_status st = check_router(r, true);
   if (st != NVFP4_OK) return st;
   if (!aligned(x, 16) || (y && !aligned(y, 16)) || (x_route && !aligned(x_route, 16))) return NVFP4_ERR_ALIGNMENT;
   const FwdLayout L = fwd_layout(T, dense);
@@ -375,12 +417,15 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const moe_experts* ex
   }
 
   ExpertArgs xa;
-  xa.gu_q = ex->gate_up_q;
-  xa.gu_s = ex->gate_up_s;
-  xa.gu_g = ex->gate_up_g;
-  xa.dn_q = ex->down_q;
-  xa.dn_s = ex->down_s;
-  xa.dn_g = ex->down_g;
+  xa.codec = ex.codec;
+  xa.gu_q = ex.gu_q;
+  xa.gu_s = ex.gu_s;
+  xa.gu_g = ex.gu_g;
+  xa.gu_b = ex.gu_b;
+  xa.dn_q = ex.dn_q;
+  xa.dn_s = ex.dn_s;
+  xa.dn_g = ex.dn_g;
+  xa.dn_b = ex.dn_b;
   xa.x = static_cast<const uint16_t*>(x);
   xa.meta = pa.meta;
   xa.sorted_slot = pa.sorted_slot;
@@ -492,7 +537,8 @@ nvfp4_status moe_block_forward(const void* x, int32_t T, const moe_block* b, voi
                            static_cast<const uint16_t*>(b->pre_ff_norm_2), b->eps, T, x1, x2, s);
   if (e != cudaSuccess) return cuda_fail(e);
   // the sparse branch: router on the raw residual, experts on x2; per-slot rows stay in ws
-  st = forward_impl(x2, T, &b->experts, &b->router, nullptr, ws, ws_bytes, stream, nullptr, false, x, false);
+  st = forward_impl(x2, T, nvfp4_ptrs(&b->experts), &b->router, nullptr, ws, ws_bytes, stream, nullptr, false, x,
+                    false);
   if (st != NVFP4_OK) return st;
   // the dense branch
   DenseArgs da;
@@ -534,7 +580,21 @@ nvfp4_status moe_block_forward(const void* x, int32_t T, const moe_block* b, voi
 
 nvfp4_status moe_nvfp4_forward(const void* x, int32_t T, const moe_experts* ex, const moe_router* r,
                                void* y, void* ws, size_t ws_bytes, void* stream) {
-  return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, nullptr);
+  const nvfp4_status st = check_experts(ex);
+  if (st != NVFP4_OK) return st;
+  return forward_impl(x, T, nvfp4_ptrs(ex), r, y, ws, ws_bytes, stream, nullptr);
+}
+
+size_t moe_aff4_forward_workspace_bytes(int32_t T, const moe_experts_aff4* ex, const moe_router* r) {
+  if (T < 1 || T > 65536 || check_experts_aff4(ex) != NVFP4_OK || check_router(r, true) != NVFP4_OK) return 0;
+  return fwd_layout(T).total;
+}
+
+nvfp4_status moe_aff4_forward(const void* x, int32_t T, const moe_experts_aff4* ex, const moe_router* r, void* y,
+                              void* ws, size_t ws_bytes, void* stream) {
+  const nvfp4_status st = check_experts_aff4(ex);
+  if (st != NVFP4_OK) return st;
+  return forward_impl(x, T, aff4_ptrs(ex), r, y, ws, ws_bytes, stream, nullptr);
 }
 
 size_t moe_forward_dense_workspace_bytes(int32_t T, const moe_experts* ex, const moe_router* r) {
@@ -545,13 +605,17 @@ size_t moe_forward_dense_workspace_bytes(int32_t T, const moe_experts* ex, const
 
 nvfp4_status moe_nvfp4_forward_dense(const void* x, int32_t T, const moe_experts* ex, const moe_router* r,
                                      void* y, void* ws, size_t ws_bytes, void* stream) {
-  return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, nullptr, true);
+  const nvfp4_status st = check_experts(ex);
+  if (st != NVFP4_OK) return st;
+  return forward_impl(x, T, nvfp4_ptrs(ex), r, y, ws, ws_bytes, stream, nullptr, true);
 }
 
 nvfp4_status moe_nvfp4_forward_profiled(const void* x, int32_t T, const moe_experts* ex,
                                         const moe_router* r, void* y, void* ws, size_t ws_bytes,
                                         void* stream, void* const* phase_events) {
-  return forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, phase_events);
+  const nvfp4_status st = check_experts(ex);
+  if (st != NVFP4_OK) return st;
+  return forward_impl(x, T, nvfp4_ptrs(ex), r, y, ws, ws_bytes, stream, phase_events);
 }
 
 nvfp4_status nvfp4_selftest_wait_timeout(const void* w, int64_t E, int64_t N, int64_t K, uint8_t* q, uint8_t* s,

@@ -29,6 +29,10 @@ constexpr int kSegK = 128;
 constexpr int kGuSegs = kH / kSegK;              // 22
 constexpr int kDnSegs = (kI + kSegK - 1) / kSegK; // 6 (the last one half full)
 
+// Expert weight codecs.
+constexpr int kCodecNvfp4 = 0;  // E2M1 codes, E4M3 scale per 16, FP32 global per expert
+constexpr int kCodecAff4 = 1;   // u4 codes, fp16 scale and bias per 32
+
 // Device status codes (mirror nvfp4_status).
 constexpr int kStatusTimeout = 5;
 constexpr int kStatusDevice = 7;
@@ -60,6 +64,31 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&o)[4]) {
       "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
       : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
       : "r"(w));
+}
+
+// Four packed bytes (eight unsigned 4-bit aff4 codes q, element 2i in the low
+// nibble of byte i) -> four f16x2 registers of q * scale + bias, register i
+// holding elements 2i (low half) and 2i+1 (high half).  Each code first
+// becomes the f16 1024 + q (q placed in the mantissa under the exponent of
+// 1024), 1024 is subtracted exactly, and one f16x2 fma applies the block's
+// scale and bias (s2, b2: each broadcast to both halves), so the weight is
+// rounded once to f16.
+__device__ __forceinline__ void u4x8_affine_f16x2(uint32_t w, uint32_t s2, uint32_t b2, uint32_t (&o)[4]) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t x01 = __byte_perm(lo, hi, 0x5140);  // elements 0, 1, 2, 3 as bytes
+  const uint32_t x23 = __byte_perm(lo, hi, 0x7362);  // elements 4, 5, 6, 7
+  const uint32_t e = 0x64646464u;                    // high byte of the f16 1024
+  uint32_t q[4];
+  q[0] = __byte_perm(x01, e, 0x4140);
+  q[1] = __byte_perm(x01, e, 0x4342);
+  q[2] = __byte_perm(x23, e, 0x4140);
+  q[3] = __byte_perm(x23, e, 0x4342);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t t;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(t) : "r"(q[i]), "r"(0x64006400u));  // exact: q
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(o[i]) : "r"(t), "r"(s2), "r"(b2));
+  }
 }
 
 // Two E4M3 bytes (low byte first) -> f16x2 (exact).

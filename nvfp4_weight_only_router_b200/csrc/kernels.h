@@ -72,12 +72,15 @@ cudaError_t launch_dense_permute(const int32_t* ids, const float* wts, int T, in
                                  int* slot_pos, float* wdense, int* status, cudaStream_t st);
 
 struct ExpertArgs {
+  int codec;                // kCodecNvfp4 or kCodecAff4
   const uint8_t* gu_q;
-  const uint8_t* gu_s;
-  const float* gu_g;
+  const uint8_t* gu_s;      // NVFP4: e4m3 [E, 2I, H/16]; aff4: fp16 scales [E, 2I, H/32]
+  const float* gu_g;        // NVFP4: FP32 global [E]; aff4: unused
+  const uint16_t* gu_b;     // aff4: fp16 biases [E, 2I, H/32]
   const uint8_t* dn_q;
   const uint8_t* dn_s;
   const float* dn_g;
+  const uint16_t* dn_b;
   const uint16_t* x;        // bf16 [T, H] (the layer input)
   __half* xs;               // [S, H] activations in expert-sorted slot order
   const int* meta;

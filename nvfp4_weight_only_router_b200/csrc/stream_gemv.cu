@@ -129,9 +129,14 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
 // (8w, 8w+1), (8w+2, 8w+3) [A0] and (8w+4, 8w+5), (8w+6, 8w+7) [A1]; the
 // activation chunk of word w (loaded from shared memory at xo ^ 16w, plus
 // 8 rows per n-tile) carries the same eight K in the same order.
-template <int NNT, int CH>
+//
+// NVFP4: sc0 / sc1 hold the two e4m3 block scales (as f16x2) of rows g and
+// g+8 for the chunk's two 16-K blocks.  aff4: the chunk is one 32-K block,
+// sc0 / sc1 its fp16 scale and bi0 / bi1 its fp16 bias (each broadcast to
+// both halves), and the weights are q * scale + bias.
+template <int NNT, int CH, int CODEC>
 __device__ __forceinline__ void mma_chunk(float (&acc)[NNT][CH][4], const uint4& w0, const uint4& w1, uint32_t sc0,
-                                          uint32_t sc1, const uint8_t* xs, uint32_t xo) {
+                                          uint32_t sc1, uint32_t bi0, uint32_t bi1, const uint8_t* xs, uint32_t xo) {
   const uint32_t a0[4] = {w0.x, w0.y, w0.z, w0.w};
   const uint32_t a1[4] = {w1.x, w1.y, w1.z, w1.w};
   const uint32_t s0lo = bcast_lo(sc0), s0hi = bcast_hi(sc0);
@@ -142,13 +147,21 @@ __device__ __forceinline__ void mma_chunk(float (&acc)[NNT][CH][4], const uint4&
 #pragma unroll
     for (int nt = 0; nt < NNT; ++nt) xb[nt] = lds_v4(xs + ((xo + nt * 8 * kXRowBytes) ^ (uint32_t)(w << 4)));
     uint32_t f0[4], f1[4];
-    e2m1x8_to_f16x2(a0[w], f0);
-    e2m1x8_to_f16x2(a1[w], f1);
-    const uint32_t s0 = w < 2 ? s0lo : s0hi, s1 = w < 2 ? s1lo : s1hi;
-    const uint32_t A0[4] = {hmul2_u32(f0[0], s0), hmul2_u32(f1[0], s1), hmul2_u32(f0[1], s0),
-                            hmul2_u32(f1[1], s1)};
-    const uint32_t A1[4] = {hmul2_u32(f0[2], s0), hmul2_u32(f1[2], s1), hmul2_u32(f0[3], s0),
-                            hmul2_u32(f1[3], s1)};
+    if (CODEC == kCodecNvfp4) {
+      e2m1x8_to_f16x2(a0[w], f0);
+      e2m1x8_to_f16x2(a1[w], f1);
+      const uint32_t s0 = w < 2 ? s0lo : s0hi, s1 = w < 2 ? s1lo : s1hi;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f0[i] = hmul2_u32(f0[i], s0);
+        f1[i] = hmul2_u32(f1[i], s1);
+      }
+    } else {
+      u4x8_affine_f16x2(a0[w], sc0, bi0, f0);
+      u4x8_affine_f16x2(a1[w], sc1, bi1, f1);
+    }
+    const uint32_t A0[4] = {f0[0], f1[0], f0[1], f1[1]};
+    const uint32_t A1[4] = {f0[2], f1[2], f0[3], f1[3]};
 #pragma unroll
     for (int nt = 0; nt < NNT; ++nt) {
       mma_f16_16816(acc[nt][w % CH], A0, xb[nt].x, xb[nt].y);
@@ -157,37 +170,61 @@ __device__ __forceinline__ void mma_chunk(float (&acc)[NNT][CH][4], const uint4&
   }
 }
 
+// A lane's block-scale words of one stage: NVFP4 .x / .y = the four e4m3
+// scales of rows A / B; aff4 also .z / .w = the rows' two fp16 biases (and
+// .x / .y their two fp16 scales).
+template <int CODEC>
+struct SWord {
+  using T = uint2;
+};
+template <>
+struct SWord<kCodecAff4> {
+  using T = uint4;
+};
+
 // The consumer's walk over its (unit, stage) sequence, used twice: once to
-// prefetch the e4m3 scales three stages ahead, once to compute.
-template <int KIND>
+// prefetch the block scales three stages ahead, once to compute.
+template <int KIND, int CODEC>
 struct ScalePrefetch {
+  using W = typename SWord<CODEC>::T;
   const int* offs;           // per-expert slot offsets (shared memory)
   const uint8_t* scales;     // gate_up or down scale matrix
+  const uint8_t* biases;     // aff4: gate_up or down bias matrix
   const int* prefix;
   int begin, n_local, rowA, rowB, q;
   int u, kc;                 // next stage to prefetch
-  const uint8_t *sa, *sb;    // scale rows of unit u
+  size_t ra, rb;             // byte offsets of the scale rows of unit u
 
   __device__ __forceinline__ void set_unit() {
     if (u >= n_local) return;
     const Unit U = decode_unit<KIND>(prefix, offs, begin + u);
     if (KIND == kGateUp) {
       const size_t g0 = (size_t)U.e * (2 * kI) + (size_t)U.j * 64;  // first gate row of the unit
-      sa = scales + (g0 + rowA) * kGuScaleRow;                      // rowA < 64: gate row
-      sb = scales + (g0 + kI + (rowB - 64)) * kGuScaleRow;          // rowB >= 64: up row
+      ra = (g0 + rowA) * kGuScaleRow;                               // rowA < 64: gate row
+      rb = (g0 + kI + (rowB - 64)) * kGuScaleRow;                   // rowB >= 64: up row
     } else {
       const size_t r0 = (size_t)U.e * kH + (size_t)U.j * kURows;
-      sa = scales + (r0 + rowA) * kDnScaleRow;
-      sb = scales + (r0 + rowB) * kDnScaleRow;
+      ra = (r0 + rowA) * kDnScaleRow;
+      rb = (r0 + rowB) * kDnScaleRow;
     }
   }
-  // scale bytes of blocks 16 kc + 4q .. +3 of both rows (the lane's 64 K of
-  // the stage); zero past the end of the unit range or of a down row
-  __device__ __forceinline__ uint2 next() {
-    uint2 v = make_uint2(0u, 0u);
+  // scale bytes [16 kc + 4q, +4) of both rows (the lane's 64 K of the stage:
+  // four e4m3 scales, or two fp16 aff4 scales and, at the same offsets, two
+  // biases); zero past the end of the unit range or of a down row
+  __device__ __forceinline__ W next() {
+    W v;
+    v.x = v.y = 0u;
+    if constexpr (CODEC == kCodecAff4) v.z = v.w = 0u;
     if (u < n_local) {
       const int b = kc * 16 + 4 * q;
-      if (KIND == kGateUp || b < kDnScaleRow) v = make_uint2(ldg_nc_u32(sa + b), ldg_nc_u32(sb + b));
+      if (KIND == kGateUp || b < kDnScaleRow) {
+        v.x = ldg_nc_u32(scales + ra + b);
+        v.y = ldg_nc_u32(scales + rb + b);
+        if constexpr (CODEC == kCodecAff4) {
+          v.z = ldg_nc_u32(biases + ra + b);
+          v.w = ldg_nc_u32(biases + rb + b);
+        }
+      }
       if (++kc == SCfg<KIND>::KC) {
         kc = 0;
         u += kGroups;
@@ -208,17 +245,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const CUtensorMap
 }
 
 // Per-lane constants of a consumer warp and its scale prefetch queue.
+template <int CODEC>
 struct Lane {
   uint32_t cA[2], cB[2];  // code byte offsets in a stage, per segment half s
   uint32_t xo[2];         // activation byte offset of chunk 8q + 4s (n-tile 0), per s
-  uint2 sq[3];            // scale words of the next three stages
+  typename SWord<CODEC>::T sq[3];  // scale words of the next three stages
 };
 
 // All stages of one unit for one consumer warp, then its epilogue.  False if
 // a wait gave up.
-template <int KIND, int NNT>
+template <int KIND, int CODEC, int NNT>
 __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, const Unit& U, int u, int n_local,
-                                             Lane& L, ScalePrefetch<KIND>& pf, int wq, int g, int q) {
+                                             Lane<CODEC>& L, ScalePrefetch<KIND, CODEC>& pf, int wq, int g, int q) {
   using C = SCfg<KIND>;
   constexpr int CH = 4 / NNT;  // independent accumulator chains per n-tile
   // the epilogue's global reads, issued now so their latency hides behind the
@@ -228,7 +266,8 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
   // (down) its routing weight, folded into one factor per column:
   //   gate_up: G_gu * 2^(e - 15) (undoes the activation prescale)
   //   down:    w * G_d * 2^(2 h_exp(e)) (undoes the hidden prescale)
-  const float G = KIND == kGateUp ? __ldg(p.gu_g + U.e) : __ldg(p.dn_g + U.e);
+  // the expert's global scale (NVFP4; aff4 has none)
+  const float G = CODEC == kCodecAff4 ? 1.0f : (KIND == kGateUp ? __ldg(p.gu_g + U.e) : __ldg(p.dn_g + U.e));
   float wgt[NNT][2];  // gate_up: G_gu * 2^(e - 15); down: w * G_d * 2^(2 h_exp(e))
   float hsc[NNT][2];  // gate_up: 2^(-2 h_exp(e))
 #pragma unroll
@@ -254,7 +293,7 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
       for (int k = 0; k < 4; ++k) acc[nt][w][k] = 0.f;
 
   for (int kc = 0; kc < C::KC; ++kc) {
-    const uint2 sq = L.sq[0];
+    const auto sq = L.sq[0];
     L.sq[0] = L.sq[1];
     L.sq[1] = L.sq[2];
     L.sq[2] = pf.next();
@@ -268,9 +307,17 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
       const uint4 w0 = lds_v4(code + L.cA[s2]);
       const uint4 w1 = lds_v4(code + L.cB[s2]);
       // blocks 2cc, 2cc+1 (cc = 2q + s2) of each row: half s2 of the lane's scale word
-      const uint32_t s0 = e4m3x2_to_f16x2((uint16_t)(s2 ? (sq.x >> 16) : (sq.x & 0xFFFFu)));
-      const uint32_t s1 = e4m3x2_to_f16x2((uint16_t)(s2 ? (sq.y >> 16) : (sq.y & 0xFFFFu)));
-      mma_chunk<NNT, CH>(acc, w0, w1, s0, s1, xs, L.xo[s2]);
+      if constexpr (CODEC == kCodecNvfp4) {
+        // blocks 2s2, 2s2+1 of the lane's four: half s2 of each row's scale word
+        const uint32_t s0 = e4m3x2_to_f16x2((uint16_t)(s2 ? (sq.x >> 16) : (sq.x & 0xFFFFu)));
+        const uint32_t s1 = e4m3x2_to_f16x2((uint16_t)(s2 ? (sq.y >> 16) : (sq.y & 0xFFFFu)));
+        mma_chunk<NNT, CH, CODEC>(acc, w0, w1, s0, s1, 0u, 0u, xs, L.xo[s2]);
+      } else {
+        // block s2 of the lane's two: half s2 of each row's scale and bias words
+        const uint32_t s0 = s2 ? bcast_hi(sq.x) : bcast_lo(sq.x), s1 = s2 ? bcast_hi(sq.y) : bcast_lo(sq.y);
+        const uint32_t b0 = s2 ? bcast_hi(sq.z) : bcast_lo(sq.z), b1 = s2 ? bcast_hi(sq.w) : bcast_lo(sq.w);
+        mma_chunk<NNT, CH, CODEC>(acc, w0, w1, s0, s1, b0, b1, xs, L.xo[s2]);
+      }
     }
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.empty[slot]);
@@ -310,7 +357,7 @@ __device__ __forceinline__ bool consume_unit(SSmem& sm, const ExpertArgs& p, con
   return true;
 }
 
-template <int KIND>
+template <int KIND, int CODEC>
 __global__ void __launch_bounds__(kThreads, 1)
     stream_gemv_kernel(const __grid_constant__ CUtensorMap tm_code, const __grid_constant__ CUtensorMap tm_x8,
                        const __grid_constant__ CUtensorMap tm_x16, ExpertArgs p) {
@@ -405,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // units 8wq..8wq+7 in rows 0..63, their up rows in 64..127)
     const int rowA = KIND == kGateUp ? 8 * wq + g : 16 * wq + g;
     const int rowB = KIND == kGateUp ? 64 + 8 * wq + g : 16 * wq + g + 8;
-    Lane L;
+    Lane<CODEC> L;
     // code chunk cc = 2q + s of rows rowA / rowB (128B swizzle: chunk ^ (row & 7) = chunk ^ g)
 #pragma unroll
     for (int s2 = 0; s2 < 2; ++s2) {
@@ -416,9 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int k = (4 * (g & 1) + q) & 7;
       L.xo[s2] = (uint32_t)(g * kXRowBytes + 128 * q + (((4 * s2) ^ k) << 4));
     }
-    ScalePrefetch<KIND> pf;
+    ScalePrefetch<KIND, CODEC> pf;
     pf.offs = sm.offs;
     pf.scales = KIND == kGateUp ? p.gu_s : p.dn_s;
+    pf.biases = reinterpret_cast<const uint8_t*>(KIND == kGateUp ? p.gu_b : p.dn_b);
     pf.prefix = sm.unit_prefix;
     pf.begin = begin;
     pf.n_local = n_local;
@@ -433,8 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     L.sq[2] = pf.next();
     for (int u = grp; u < n_local; u += kGroups) {
       const Unit U = decode_unit<KIND>(sm.unit_prefix, sm.offs, begin + u);
-      const bool ok = U.nvalid > 8 ? consume_unit<KIND, 2>(sm, p, U, u, n_local, L, pf, wq, g, q)
-                                   : consume_unit<KIND, 1>(sm, p, U, u, n_local, L, pf, wq, g, q);
+      const bool ok = U.nvalid > 8 ? consume_unit<KIND, CODEC, 2>(sm, p, U, u, n_local, L, pf, wq, g, q)
+                                   : consume_unit<KIND, CODEC, 1>(sm, p, U, u, n_local, L, pf, wq, g, q);
       if (!ok) break;
     }
   }
@@ -449,11 +497,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 }
 
-template <int KIND>
+template <int KIND, int CODEC>
 cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t st) {
   using C = SCfg<KIND>;
   const int smem = (int)sizeof(SSmem) + 1024;  // + alignment slack
-  cudaError_t err = configure_kernel_once((const void*)stream_gemv_kernel<KIND>, smem);
+  cudaError_t err = configure_kernel_once((const void*)stream_gemv_kernel<KIND, CODEC>, smem);
   if (err != cudaSuccess) return err;
   CUtensorMap tm_code;
   bool ok;
@@ -486,7 +534,7 @@ cudaError_t launch_stream(const ExpertArgs& a, cudaStream_t st) {
   int sms = 0;
   err = sm_count(&sms);
   if (err != cudaSuccess) return err;
-  stream_gemv_kernel<KIND><<<sms, kThreads, smem, st>>>(tm_code, tm_x8, tm_x16, a);
+  stream_gemv_kernel<KIND, CODEC><<<sms, kThreads, smem, st>>>(tm_code, tm_x8, tm_x16, a);
   return cudaGetLastError();
 }
 
@@ -494,7 +542,11 @@ static_assert(sizeof(SSmem) + 1024 <= 232448, "shared memory budget");
 
 }  // namespace
 
-cudaError_t launch_gate_up_stream(const ExpertArgs& a, cudaStream_t st) { return launch_stream<kGateUp>(a, st); }
-cudaError_t launch_down_stream(const ExpertArgs& a, cudaStream_t st) { return launch_stream<kDown>(a, st); }
+cudaError_t launch_gate_up_stream(const ExpertArgs& a, cudaStream_t st) {
+  return a.codec == kCodecAff4 ? launch_stream<kGateUp, kCodecAff4>(a, st) : launch_stream<kGateUp, kCodecNvfp4>(a, st);
+}
+cudaError_t launch_down_stream(const ExpertArgs& a, cudaStream_t st) {
+  return a.codec == kCodecAff4 ? launch_stream<kDown, kCodecAff4>(a, st) : launch_stream<kDown, kCodecNvfp4>(a, st);
+}
 
 }  // namespace nvfp4moe

@@ -168,7 +168,7 @@ __device__ __forceinline__ void tc_commit_warp(uint64_t* bar) {
       : "memory");
 }
 
-template <int KIND, int NT>
+template <int KIND, int NT, int CODEC>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_moe_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                   ExpertArgs p) {
@@ -257,19 +257,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int L = quarter * 32 + lane;  // tensor-memory lane = A row
     // code / scale row in shared memory: gate_up stores gate rows 0..63 then up rows 64..127
     const int crow = KIND == kGateUp ? ((L & 1) * 64 + (L >> 1)) : L;
-    // this lane's e4m3 scale pair of each chunk, read from global memory
-    // three chunks ahead of its use (the walk crosses tile boundaries)
+    // this lane's block scales of each chunk, read from global memory three
+    // chunks ahead of its use (the walk crosses tile boundaries): NVFP4, the
+    // two e4m3 scales of its 32 K; aff4, the one fp16 scale and (high half)
+    // fp16 bias of its 32 K, which sit at the same byte offsets
     const uint8_t* sc_src = KIND == kGateUp ? p.gu_s : p.dn_s;
+    const uint8_t* bi_src = reinterpret_cast<const uint8_t*>(KIND == kGateUp ? p.gu_b : p.dn_b);
     int pt = blockIdx.x, pkc = 0;
-    const uint8_t* prow = nullptr;
-    auto prow_of = [&](int t) -> const uint8_t* {
+    size_t prow = 0;
+    auto prow_of = [&](int t) -> size_t {
       const TileInfo ti = decode_tile<KIND, NT>(sm, p.meta, t);
-      return sc_src + (size_t)tile_row<KIND>(ti.e, ti.j, L) * C::SROW + khalf * 2;
+      return (size_t)tile_row<KIND>(ti.e, ti.j, L) * C::SROW + khalf * 2;
     };
     if (pt < n_tiles) prow = prow_of(pt);
-    auto next_scale = [&]() -> uint16_t {
+    auto next_scale = [&]() -> uint32_t {
       if (pt >= n_tiles) return 0;
-      const uint16_t v = ldg_nc_u16(prow + pkc * 4);
+      uint32_t v = ldg_nc_u16(sc_src + prow + pkc * 4);
+      if (CODEC == kCodecAff4) v |= (uint32_t)ldg_nc_u16(bi_src + prow + pkc * 4) << 16;
       if (++pkc == C::KC) {
         pkc = 0;
         pt += gridDim.x;
@@ -277,14 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       return v;
     };
-    uint16_t sq0 = next_scale(), sq1 = next_scale(), sq2 = next_scale();
+    uint32_t sq0 = next_scale(), sq1 = next_scale(), sq2 = next_scale();
     uint32_t kiter = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
       for (int kc = 0; kc < C::KC; ++kc, ++kiter) {
         const int s = kiter % C::NS, use = kiter / C::NS;
         const int a = kiter % C::NA, ause = kiter / C::NA;
-        const uint16_t sq = sq0;
+        const uint32_t sq = sq0;
         sq0 = sq1;
         sq1 = sq2;
         sq2 = next_scale();
@@ -295,17 +299,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint4 w = lds_v4(sm.code[s] + crow * 32 + khalf * 16);   // 32 K of this row
-        const uint32_t s2 = e4m3x2_to_f16x2(sq);
-        const uint32_t slo = bcast_lo(s2), shi = bcast_hi(s2);
         const uint32_t words[4] = {w.x, w.y, w.z, w.w};
         uint32_t v[16];
+        if (CODEC == kCodecNvfp4) {
+          const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)sq);
+          const uint32_t slo = bcast_lo(s2), shi = bcast_hi(s2);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t f[4];
-          e2m1x8_to_f16x2(words[q], f);
-          const uint32_t scl = q < 2 ? slo : shi;
+          for (int q = 0; q < 4; ++q) {
+            uint32_t f[4];
+            e2m1x8_to_f16x2(words[q], f);
+            const uint32_t scl = q < 2 ? slo : shi;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) v[4 * q + i] = hmul2_u32(f[i], scl);
+            for (int i = 0; i < 4; ++i) v[4 * q + i] = hmul2_u32(f[i], scl);
+          }
+        } else {
+          const uint32_t scl = bcast_lo(sq), bia = bcast_hi(sq);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t f[4];
+            u4x8_affine_f16x2(words[q], scl, bia, f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[4 * q + i] = f[i];
+          }
         }
         tmem_st16(taddr + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(C::A_COL0 + a * 32 + khalf * 16), v);
         tmem_wait_st();
@@ -385,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           slot[i] = (KIND == kDown && n < nvalid) ? __ldg(p.sorted_slot + pos0 + n) : -1;
         }
         if (KIND == kDown) {
-          const float G = p.dn_g[ti.e];
+          const float G = CODEC == kCodecAff4 ? 1.0f : p.dn_g[ti.e];
           float wv[PER];
 #pragma unroll
           for (int i = 0; i < PER; ++i) wv[i] = slot[i] >= 0 ? __ldg(p.wts + slot[i]) : 0.f;
@@ -407,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lane pair (2r, 2r+1) = (gate, up) of hidden unit 16*quarter + r of the
         // tile; h values go to this warp's staging [token][16 units] and leave
         // as 32-byte row pieces (two lanes per token row)
-        const float G = p.gu_g[ti.e];
+        const float G = CODEC == kCodecAff4 ? 1.0f : p.gu_g[ti.e];
         const bool odd = L & 1;
         const int ul = lane >> 1;  // unit within the warp's 16
         bool over = false;
@@ -492,10 +507,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 static_assert(sizeof(MoeSmem<kGateUp, 192>) + 1024 <= 232448, "shared memory budget (gate_up)");
 static_assert(sizeof(MoeSmem<kDown, 192>) + 1024 <= 232448, "shared memory budget (down)");
 
-template <int KIND, int NT>
+template <int KIND, int NT, int CODEC>
 cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
   const int smem = (int)sizeof(MoeSmem<KIND, NT>) + 1024;  // + alignment slack
-  cudaError_t err = configure_kernel_once((const void*)tc_moe_kernel<KIND, NT>, smem);
+  cudaError_t err = configure_kernel_once((const void*)tc_moe_kernel<KIND, NT, CODEC>, smem);
   if (err != cudaSuccess) return err;
   const uint64_t S = (uint64_t)a.T * a.spt;
   CUtensorMap tm_x, tm_w;
@@ -513,7 +528,7 @@ cudaError_t launch_moe(const ExpertArgs& a, cudaStream_t st) {
   int sms = 0;
   err = sm_count(&sms);
   if (err != cudaSuccess) return err;
-  tc_moe_kernel<KIND, NT><<<sms, kThreads, smem, st>>>(tm_x, tm_w, a);
+  tc_moe_kernel<KIND, NT, CODEC><<<sms, kThreads, smem, st>>>(tm_x, tm_w, a);
   return cudaGetLastError();
 }
 
@@ -584,20 +599,23 @@ cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_moe_gate_up(const ExpertArgs& a, int nt, cudaStream_t st) {
+template <int KIND, int CODEC>
+cudaError_t launch_moe_nt(const ExpertArgs& a, int nt, cudaStream_t st) {
   switch (nt) {
-    case 16: return launch_moe<kGateUp, 16>(a, st);
-    case 64: return launch_moe<kGateUp, 64>(a, st);
-    default: return launch_moe<kGateUp, 192>(a, st);
+    case 16: return launch_moe<KIND, 16, CODEC>(a, st);
+    case 64: return launch_moe<KIND, 64, CODEC>(a, st);
+    default: return launch_moe<KIND, 192, CODEC>(a, st);
   }
 }
 
+cudaError_t launch_moe_gate_up(const ExpertArgs& a, int nt, cudaStream_t st) {
+  return a.codec == kCodecAff4 ? launch_moe_nt<kGateUp, kCodecAff4>(a, nt, st)
+                               : launch_moe_nt<kGateUp, kCodecNvfp4>(a, nt, st);
+}
+
 cudaError_t launch_moe_down(const ExpertArgs& a, int nt, cudaStream_t st) {
-  switch (nt) {
-    case 16: return launch_moe<kDown, 16>(a, st);
-    case 64: return launch_moe<kDown, 64>(a, st);
-    default: return launch_moe<kDown, 192>(a, st);
-  }
+  return a.codec == kCodecAff4 ? launch_moe_nt<kDown, kCodecAff4>(a, nt, st)
+                               : launch_moe_nt<kDown, kCodecNvfp4>(a, nt, st);
 }
 
 }  // namespace nvfp4moe

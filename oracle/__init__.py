@@ -27,10 +27,13 @@ Sources (page title, section):
     a dense GELU-gated MLP (intermediate 2112) in parallel with the sparse
     branch, five norms, the router on the raw residual, and layer_scalar.
 
+  * The same card's "Compression recipe", for the aff4 codec (oracle/aff4):
+    affine int4 with an fp16 scale and bias per (row, K-block of 32).
+
 Parity pins: every function here is pinned by a `-m "not gpu"` test against
 closed forms, library routines (torch float8_e4m3fn, torch softmax/gelu/rms_norm,
 numpy matmul), exhaustive enumeration or brute force on tiny inputs.  The
 pages' own verification numbers need trained weights that are not available,
 so the forward pass is pinned by invariants and brute force only.
 """
-from . import formats, quantize, moe, block  # noqa: F401
+from . import formats, quantize, moe, block, aff4  # noqa: F401

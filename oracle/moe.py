@@ -103,7 +103,12 @@ def gelu_tanh(g: np.ndarray) -> np.ndarray:
 
 
 def expert_dense(experts, e: int):
-    """Float64 dequantised weights of expert e: (W_gate_up [2I, H], W_down [H, I])."""
+    """Float64 dequantised weights of expert e: (W_gate_up [2I, H], W_down [H, I]).
+    NVFP4 experts here; experts of the aff4 codec dequantise through
+    oracle/aff4.py."""
+    if getattr(experts, "codec", "nvfp4") == "aff4":
+        from . import aff4
+        return aff4.expert_dense(experts, e)
     wgu = dequantize(experts.gate_up_q[e], experts.gate_up_s[e], experts.gate_up_g[e])
     wd = dequantize(experts.down_q[e], experts.down_s[e], experts.down_g[e])
     return wgu, wd

@@ -25,7 +25,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported(capi):
     names = header_functions()
-    assert len(names) == 22
+    assert len(names) == 24
     for n in names:
         assert hasattr(capi.lib, n), n
         assert n in capi.SIGNATURES, n
@@ -200,3 +200,20 @@ def test_block_validation(capi):
     assert c.moe_block_forward(P, 1, ctypes.byref(bad), P, P, ws, None) == c.NVFP4_ERR_ALIGNMENT
     bad.post_ff_norm = None
     assert c.moe_block_forward(P, 1, ctypes.byref(bad), P, P, ws, None) == c.NVFP4_ERR_INVALID_ARG
+
+
+def test_aff4_validation(capi):
+    c = capi
+    r = _router(c)
+    a = c.moe_experts_aff4(4096, 4096, 4096, 4096, 4096, 4096, 128, 2816, 704)
+    x = _experts(c)
+    n = c.moe_aff4_forward_workspace_bytes(64, ctypes.byref(a), ctypes.byref(r))
+    assert n == c.moe_forward_workspace_bytes(64, ctypes.byref(x), ctypes.byref(r))   # the same layout
+    P = 4096
+    bad = c.moe_experts_aff4(4096, 4096, None, 4096, 4096, 4096, 128, 2816, 704)
+    assert c.moe_aff4_forward(P, 1, ctypes.byref(bad), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_INVALID_ARG
+    bad = c.moe_experts_aff4(4096, 4096, 4096, 4096, 4096, 4096, 128, 2816, 512)
+    assert c.moe_aff4_forward(P, 1, ctypes.byref(bad), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_UNSUPPORTED
+    bad = c.moe_experts_aff4(4096, 4096 + 2, 4096, 4096, 4096, 4096, 128, 2816, 704)
+    assert c.moe_aff4_forward(P, 1, ctypes.byref(bad), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_ALIGNMENT
+    assert c.moe_aff4_forward(P, 1, ctypes.byref(a), ctypes.byref(r), P, P, 0, None) == c.NVFP4_ERR_WORKSPACE
