@@ -118,8 +118,8 @@ typedef struct {
  * Workspace: nvfp4_quantize_workspace_bytes(E, N, K) bytes, 256-aligned
  * (E amax words and three arrival counters; the call clears what it uses).
  * Execution: when one tensor's share per SM fits on chip (N * K / 16 blocks
- * of 32 bytes split over all SMs, at most 54 KB each, and at least 8 blocks
- * per SM) the call is one cooperative launch of one CTA per SM that reads
+ * of 32 bytes split over all SMs, at most 1700 blocks each, and at least 8
+ * blocks per SM) the call is one cooperative launch of one CTA per SM that reads
  * every weight once; it occupies the whole GPU while it runs (if the
  * context cannot hold one CTA on every SM at once, the call takes the two
  * passes instead).  Other shapes take two passes (amax, then encode).  Both

@@ -140,16 +140,33 @@ __device__ __forceinline__ TensorScale tensor_scale(float amax) {
 // when both ends round to the same code, so does the exact quotient.  Where
 // they differ (a quotient within ~2^-20 of a rounding threshold) the block
 // takes the correctly rounded divisions.
-__device__ __forceinline__ uint32_t encode_block16(const uint32_t (&pair)[8], const TensorScale& ts, uint2& codes) {
-  float x[16];
+// max |w| of a block as a bf16 bit pattern (a monotone key for finite values)
+__device__ __forceinline__ uint32_t block_key16(const uint32_t (&pair)[8]) {
   uint32_t key2 = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) key2 = __vmaxu2(key2, pair[j] & 0x7FFF7FFFu);
+  return max(key2 & 0xFFFFu, key2 >> 16);
+}
+
+// two fp32 products a * r of a pair in one packed instruction (each lane
+// correctly rounded, as two separate multiplies)
+__device__ __forceinline__ void mul_f32x2(float a0, float a1, float r, float& p0, float& p1) {
+  uint64_t x, rr, out;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(rr) : "f"(r));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(out) : "l"(x), "l"(rr));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(p0), "=f"(p1) : "l"(out));
+}
+
+// encode_block16 with the block's max |w| key already known
+__device__ __forceinline__ uint32_t encode_block16k(const uint32_t (&pair)[8], uint32_t key, const TensorScale& ts,
+                                                    uint2& codes) {
+  float x[16];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     x[2 * j] = bf16_bits_to_f32(pair[j] & 0xFFFFu);
     x[2 * j + 1] = __uint_as_float(pair[j] & 0xFFFF0000u);
-    key2 = __vmaxu2(key2, pair[j] & 0x7FFF7FFFu);
   }
-  const uint32_t key = max(key2 & 0xFFFFu, key2 >> 16);
   const float amax_b = __uint_as_float(key << 16);
   const float G = ts.G;
   uint32_t sc = 0;
@@ -179,9 +196,9 @@ __device__ __forceinline__ uint32_t encode_block16(const uint32_t (&pair)[8], co
       for (int h = 0; h < 2; ++h) {
         float a[8], b[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          a[i] = __fmul_rn(x[8 * h + i], rl);
-          b[i] = __fmul_rn(x[8 * h + i], rh);
+        for (int i = 0; i < 8; i += 2) {
+          mul_f32x2(x[8 * h + i], x[8 * h + i + 1], rl, a[i], a[i + 1]);
+          mul_f32x2(x[8 * h + i], x[8 * h + i + 1], rh, b[i], b[i + 1]);
         }
         packed[h] = e2m1x8_rne(a);
         hi[h] = e2m1x8_rne(b);
@@ -205,6 +222,10 @@ __device__ __forceinline__ uint32_t encode_block16(const uint32_t (&pair)[8], co
   }
   codes = make_uint2(packed[0], packed[1]);
   return sc;
+}
+
+__device__ __forceinline__ uint32_t encode_block16(const uint32_t (&pair)[8], const TensorScale& ts, uint2& codes) {
+  return encode_block16k(pair, block_key16(pair), ts, codes);
 }
 
 __global__ void __launch_bounds__(256) encode_kernel(const uint16_t* __restrict__ w,
@@ -232,7 +253,8 @@ constexpr int kQThreads = 1024;                // warp 0: control; warps 1..31: 
 constexpr int kQCompute = kQThreads - 32;
 constexpr int kQBufs = 4;                      // tensors e (encoding), e+1, e+2 (reduced), e+3 (loading)
 constexpr int kQHeader = 1024;                 // barriers, reduction slots, tensor constants, flags
-constexpr int kQMaxPiece = 54 * 1024;          // bytes per buffer (1728 blocks)
+constexpr int kQMaxPiece = 54400;              // bytes per buffer (1700 blocks)
+constexpr int kQKeys = kQMaxPiece / 32;         // per-block max |w| keys (u16) per buffer
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
@@ -276,6 +298,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   TensorScale* ts_sh = reinterpret_cast<TensorScale*>(qsm + 128 + kQBufs * 128);  // [kQBufs]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(qsm + 960);
   uint8_t* buf0 = qsm + kQHeader;
+  uint16_t* keys = reinterpret_cast<uint16_t*>(buf0 + (size_t)kQBufs * kQMaxPiece);  // [kQBufs][kQKeys]
   uint32_t* ctr = amax_ws + E;
   const int n = gridDim.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t b0 = (int64_t)blockIdx.x * bpe / n, b1 = (int64_t)(blockIdx.x + 1) * bpe / n;
@@ -362,17 +385,21 @@ __global__ void __launch_bounds__(kQThreads, 1)
   } else {
     // ------------------------------------------------------------ compute
     const int ct = tid - 32, cw = warp - 1;
-    auto reduce = [&](int t) -> bool {  // |w| over tensor t's piece -> red[t % 4][cw]
+    // |w| over tensor t's piece -> red[t % 4][cw]; each block's own maximum
+    // is kept in keys[] for the encoder
+    auto reduce = [&](int t) -> bool {
       const int b = t % kQBufs;
       if (!mbar_wait_bounded(&full[b], (t / kQBufs) & 1, wait_ns)) return false;
       const uint4* v = reinterpret_cast<const uint4*>(buf0 + (size_t)b * kQMaxPiece);
+      uint16_t* kb = keys + (size_t)b * kQKeys;
       uint32_t m = 0;
-      for (int i = ct; i < nb * 2; i += kQCompute) {
-        const uint4 u = v[i];
-        m = __vmaxu2(m, __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
-                                 __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu)));
+      for (int lb = ct; lb < nb; lb += kQCompute) {
+        const uint4 v0 = v[2 * lb], v1 = v[2 * lb + 1];
+        const uint32_t pair[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint32_t key = block_key16(pair);
+        kb[lb] = (uint16_t)key;
+        m = max(m, key);
       }
-      m = max(m & 0xFFFFu, m >> 16);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
       if (lane == 0) {
@@ -394,12 +421,13 @@ __global__ void __launch_bounds__(kQThreads, 1)
       }
       const TensorScale ts = ts_sh[b];
       const uint4* v = reinterpret_cast<const uint4*>(buf0 + (size_t)b * kQMaxPiece);
+      const uint16_t* kb = keys + (size_t)b * kQKeys;
       const size_t gb0 = (size_t)e * bpe + b0;
       for (int lb = ct; lb < nb; lb += kQCompute) {
         const uint4 v0 = v[2 * lb], v1 = v[2 * lb + 1];
         const uint32_t pair[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         uint2 codes;
-        const uint32_t sc = encode_block16(pair, ts, codes);
+        const uint32_t sc = encode_block16k(pair, kb[lb], ts, codes);
         *reinterpret_cast<uint2*>(q + (gb0 + lb) * 8) = codes;
         s[gb0 + lb] = (uint8_t)sc;
       }
@@ -443,7 +471,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
 
 namespace {
 
-constexpr int kQSmem = kQHeader + kQBufs * kQMaxPiece;
+constexpr int kQSmem = kQHeader + kQBufs * kQMaxPiece + kQBufs * kQKeys * 2;
 static_assert(kQSmem <= 232448, "shared memory budget of the single-pass quantiser");
 
 // the single-pass kernel applies: the largest piece fits a buffer, every CTA
