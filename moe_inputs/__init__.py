@@ -175,6 +175,14 @@ def make_quant_weights(seed: int, e: int, n: int, k: int, outlier_frac: float = 
     return out
 
 
+# Static input globals of the W4A4 form (the checkpoint's per-projection
+# `input_scale`): amax / (6 * 448) for an activation range of 8 for the
+# experts' input x ~ N(0, 1) and 2 for the gated hidden of these synthetic
+# experts (|h| stays below 0.7 on seeded draws).  Inputs, not results.
+W4A4_GX = np.float32(8.0 / 2688.0)
+W4A4_GH = np.float32(2.0 / 2688.0)
+
+
 def layer_seed_plan(n_layers: int = 30, base: int = 100) -> list[int]:
     """Seeds of an independently seeded layer stack (layer l uses base + l)."""
     return [base + l for l in range(n_layers)]

@@ -36,4 +36,4 @@ numpy matmul), exhaustive enumeration or brute force on tiny inputs.  The
 pages' own verification numbers need trained weights that are not available,
 so the forward pass is pinned by invariants and brute force only.
 """
-from . import formats, quantize, moe, block, aff4  # noqa: F401
+from . import formats, quantize, moe, block, aff4, w4a4  # noqa: F401

@@ -43,15 +43,16 @@ def global_scale(w32: np.ndarray) -> np.float32:
     return np.float32(np.float32(amax) / GLOBAL_DENOM)
 
 
-def quantize_tensor(w_bits: np.ndarray):
-    """Quantise one bf16 tensor [N, K] (bf16 bit patterns) with its own
-    global scale.  Returns (packed uint8 [N, K/2], scales uint8 [N, K/16],
-    G float32)."""
-    w = bf16_to_f32(w_bits)
+def quantize_blocks(w: np.ndarray, G) -> tuple[np.ndarray, np.ndarray]:
+    """The block and element steps for float32 values w [N, K] under a given
+    FP32 global scale G: returns (packed uint8 [N, K/2], scales uint8 [N, K/16]).
+    Weights take G from their own amax (quantize_tensor); activations of the
+    W4A4 form take a static per-projection G (oracle/w4a4.py)."""
+    w = np.asarray(w, np.float32)
+    G = np.float32(G)
     n, k = w.shape
     if k % BLOCK:
         raise ValueError("K must be a multiple of 16")
-    G = global_scale(w)
     blocks = w.reshape(n, k // BLOCK, BLOCK)
     amax_b = np.max(np.abs(blocks), axis=-1)                      # float32, exact
     if G > 0:
@@ -68,7 +69,19 @@ def quantize_tensor(w_bits: np.ndarray):
     degenerate = (d == 0)[..., None] & np.ones_like(codes, dtype=bool)
     sign_only = (np.signbit(blocks).astype(np.uint8) << 3)
     codes = np.where(degenerate, sign_only, codes)
-    return pack_nibbles(codes.reshape(n, k)), s, np.float32(G)
+    return pack_nibbles(codes.reshape(n, k)), s
+
+
+def quantize_tensor(w_bits: np.ndarray):
+    """Quantise one bf16 tensor [N, K] (bf16 bit patterns) with its own
+    global scale.  Returns (packed uint8 [N, K/2], scales uint8 [N, K/16],
+    G float32)."""
+    w = bf16_to_f32(w_bits)
+    if w.shape[1] % BLOCK:
+        raise ValueError("K must be a multiple of 16")
+    G = global_scale(w)
+    q, s = quantize_blocks(w, G)
+    return q, s, np.float32(G)
 
 
 def quantize(w_bits: np.ndarray):
