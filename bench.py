@@ -77,6 +77,10 @@ WORKLOADS = {
                     "desc": "one MoE layer, prefill T=4096, Zipf(1.1)-skewed router bias"},
     "aff4_64": {"T": 64, "layers": 1, "zipf": False, "aff4": True,
                 "desc": "one MoE layer with aff4 experts (u4, fp16 scale+bias per 32), decode T=64"},
+    "w4a4_64": {"T": 64, "layers": 1, "zipf": False, "w4a4": True,
+                "desc": "one MoE layer in the W4A4 form (NVFP4 activations, block-scaled FP4 tensor cores), decode T=64"},
+    "w4a4_4096": {"T": 4096, "layers": 1, "zipf": True, "w4a4": True,
+                  "desc": "one MoE layer in the W4A4 form, prefill T=4096, Zipf(1.1)-skewed router bias"},
     "dense1": {"T": 1, "layers": 1, "zipf": False, "dense": True,
                "desc": "one MoE layer, decode T=1, dense over-read: all 128 experts per token (ablation)"},
     "block64": {"T": 64, "layers": 1, "zipf": False, "block": True,
@@ -186,8 +190,9 @@ class OracleSample:
             self.block = B.BlockParams(self.ex, self.rt, b.dense_gate, b.dense_up, b.dense_down, b.pre_ff_norm,
                                        b.post_ff_norm_1, b.pre_ff_norm_2, b.post_ff_norm_2, b.post_ff_norm,
                                        b.layer_scalar)
+        self.w4a4 = bool(wl.get("w4a4"))
         self.what = (f"oracle fp64 forward of {tokens} of the workload's tokens through one "
-                     + ("full block" if self.block else "layer"))
+                     + ("full block" if self.block else ("W4A4 layer" if self.w4a4 else "layer")))
 
     def run(self):
         """Returns (value, unit, seconds)."""
@@ -202,6 +207,10 @@ class OracleSample:
         if self.block is not None:
             from oracle import block as B
             B.forward(self.x, self.block)
+        elif self.w4a4:
+            import moe_inputs as gen
+            from oracle import w4a4 as W
+            W.forward(self.x, self.ex, self.rt, gen.W4A4_GX, gen.W4A4_GH)
         else:
             M.forward(self.x, self.ex, self.rt)
         dt = time.perf_counter() - t0
@@ -211,7 +220,7 @@ class OracleSample:
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return
-    tokens = 2 if args.workload != "prefill4096" else 4
+    tokens = 4 if args.workload in ("prefill4096", "w4a4_4096") else 2
     sample = OracleSample(args.workload, wl, tokens)
     what = sample.what
     for _ in range(min(args.warmup, 1)):
@@ -341,6 +350,9 @@ def measure(ctx, workload, args, cpu_baseline=True):
             if wl.get("block"):
                 parts = lib.DenseParts.from_host(gen.make_block(200), dev)
                 layers.append(lib.MoeBlock(ctx.experts(sd), lib.Router.from_host(rt, dev), parts, max_tokens=T))
+            elif wl.get("w4a4"):
+                layers.append(lib.W4A4Layer(ctx.experts(sd), lib.Router.from_host(rt, dev), gen.W4A4_GX, gen.W4A4_GH,
+                                            max_tokens=T))
             elif wl.get("aff4"):
                 layers.append(lib.Aff4Layer(lib.Aff4Experts.from_host(gen.make_aff4_experts(9), dev),
                                             lib.Router.from_host(rt, dev), max_tokens=T))
@@ -361,6 +373,11 @@ def measure(ctx, workload, args, cpu_baseline=True):
                 layer.forward_dense_into(xin, yout)
             elif wl.get("block") or wl.get("aff4"):
                 layer.forward_into(xin, yout)
+            elif profiled and wl.get("w4a4"):
+                arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+                capi.check(capi.moe_w4a4_forward_profiled(
+                    xin.data_ptr(), T, ctypes.byref(layer._xs), ctypes.byref(layer._rs), yout.data_ptr(),
+                    layer.workspace.data_ptr(), layer.workspace.numel(), st, arr))
             elif profiled:
                 arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
                 capi.check(capi.moe_nvfp4_forward_profiled(
@@ -534,7 +551,21 @@ def measure(ctx, workload, args, cpu_baseline=True):
         gu_ms = ph[:, 2]
         dense_bytes = 3 * 2816 * 2112 * 2
         dense_flops = 2.0 * T * 3 * 2816 * 2112
-        if wl.get("block") and T >= 1024:
+        if wl.get("w4a4") and T >= 1024:
+            # FP4 x FP4 on the tensor cores: the burst bf16 peak x the nominal fp4 / bf16 ratio (9 / 2.25)
+            ach = gu_flops / (gu_ms.mean() / 1e3) / 1e12
+            roof = {"bound": "tensor", "kernel": "gate_up W4A4 grouped GEMM + GELU + hidden quantisation (tcgen05 mxf4nvf4)",
+                    "achieved": ach, "peak": ctx.tc_peak * 4.0, "unit": "TFLOP/s", "traffic": traffic,
+                    "peak_kind": ctx.peak_kind + " burst bf16 x 4 (nominal fp4/bf16)",
+                    "algorithmic_per_launch": gu_flops}
+        elif wl.get("w4a4"):
+            # weights + the slots' activation codes and scales in, hidden codes and scales out
+            w4_bytes = n_act * GU_EXPERT_BYTES + S * (1408 + 176) + S * (352 + 44)
+            ach = w4_bytes.sum() / (gu_ms.sum() / 1e3) / 1e9
+            roof = {"bound": "hbm", "kernel": "gate_up W4A4 grouped GEMM + GELU + hidden quantisation (tcgen05 mxf4nvf4)",
+                    "achieved": ach, "peak": ctx.hbm_peak, "unit": "GB/s", "traffic": traffic,
+                    "peak_kind": ctx.peak_kind, "algorithmic_per_launch": float(w4_bytes.mean())}
+        elif wl.get("block") and T >= 1024:
             flops = 2.0 * S * (1408 * 2816 + 2816 * 704) + dense_flops
             ach = flops / (ms_per_step / 1e3) / 1e12
             roof = {"bound": "tensor", "kernel": "whole block step (experts + dense MLP, no phase split)",
@@ -581,13 +612,13 @@ def measure(ctx, workload, args, cpu_baseline=True):
             "step_hbm_gbs": float(step_bytes.mean() * wl["layers"] / (ms_per_step / 1e3) / 1e9),
             "layer_tflops": float(2.0 * S * (1408 * 2816 + 2816 * 704) * wl["layers"] / (ms_per_step / 1e3) / 1e12),
         }
-        dtype = "f16xe2m1"
+        dtype = "e2m1xe2m1" if wl.get("w4a4") else "f16xe2m1"
     if traffic_kernel:
         roof["traffic_kernel"] = traffic_kernel
 
     cpu = None
     if rank == 0 and cpu_baseline:
-        tokens = 2 if workload != "prefill4096" else 4
+        tokens = 4 if workload in ("prefill4096", "w4a4_4096") else 2
         sample = OracleSample(workload, wl, tokens)
         v, u, dt = sample.run()
         what = sample.what

@@ -324,6 +324,88 @@ NVFP4MOE_API nvfp4_status moe_block_forward(const void* x_dev, int32_t T, const 
                                             void* ws_dev, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * W4A4: the routed experts with NVFP4 activations on the block-scaled FP4
+ * tensor cores ("Gemma-4-26B-A4B-it-NVFP4": built for native FP4 tensor-core
+ * execution, block-scale formulas; "Gemma-4-26B-A4B-NVFP4-mlx": the
+ * checkpoint's `input_scale` sidecar, a static FP32 global per projection
+ * input; "gemma-4-26B-A4B . NVFP4A16": W4A16 keeps BF16 activations and
+ * forgoes this form's activation speed-up).
+ * Each token's x is quantised once as a weight row is (blocks of 16 along H,
+ * E4M3 scale s = e4m3_rn_satfinite((amax_b / 6) / Gx), E2M1 codes of x / (s Gx),
+ * every step one correctly rounded fp32 operation) under the static global
+ * Gx = input_scale_gate_up; per expert the gate_up GEMM multiplies the E2M1
+ * codes of both operands with their E4M3 scales in the tensor core (fp32
+ * accumulation), h = gelu_tanh(Gx G_gu g) * (Gx G_gu u) in fp32 is quantised
+ * the same way per 16 hidden units under Gh = input_scale_down, the down GEMM
+ * multiplies those codes with the down weights', o = w G_d Gh acc per slot,
+ * and y[t] = bf16(sum over the token's 8 slots in slot order).
+ *
+ * The weights are those of moe_experts, plus their block scales copied once
+ * into the order the tensor core reads them (moe_w4a4_pack_scales): per
+ * expert, per 128-row tile of the projection and per 64 elements of K, one
+ * 512-byte chunk.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  moe_experts experts;           /* codes, block scales and globals (moe_nvfp4_forward's) */
+  const uint8_t* gate_up_sf;     /* moe_w4a4_scale_bytes(E, 0) bytes from moe_w4a4_pack_scales */
+  const uint8_t* down_sf;        /* moe_w4a4_scale_bytes(E, 1) bytes */
+  float input_scale_gate_up;     /* Gx > 0, finite */
+  float input_scale_down;        /* Gh > 0, finite */
+} moe_experts_w4a4;
+
+/* Bytes of the packed block scales of the gate_up (which = 0) or down
+ * (which = 1) projections of E experts: E * N * K / 16 (0 for E < 1 or another
+ * `which`). */
+NVFP4MOE_API size_t moe_w4a4_scale_bytes(int32_t E, int32_t which);
+
+/* moe_w4a4_pack_scales: copies experts->gate_up_s and down_s into the tensor
+ * core's order, gate_up_sf_dev / down_sf_dev of moe_w4a4_scale_bytes(E, 0/1)
+ * bytes (device, 16-byte aligned, caller-owned).  Run once per set of
+ * weights; asynchronous on `stream`.  Same shape requirements as
+ * moe_nvfp4_forward. */
+NVFP4MOE_API nvfp4_status moe_w4a4_pack_scales(const moe_experts* experts, uint8_t* gate_up_sf_dev,
+                                               uint8_t* down_sf_dev, void* stream);
+
+/* moe_w4a4_forward: y_dev bf16 [T, H] from x_dev bf16 [T, H] as described
+ * above; 1 <= T <= 65536, router and experts as for moe_nvfp4_forward.
+ * Workspace: moe_w4a4_workspace_bytes(T, experts, router) bytes, 256-byte
+ * aligned, caller-owned.  Errors as for moe_nvfp4_forward. */
+NVFP4MOE_API size_t moe_w4a4_workspace_bytes(int32_t T, const moe_experts_w4a4* experts, const moe_router* router);
+NVFP4MOE_API nvfp4_status moe_w4a4_forward(const void* x_dev, int32_t T, const moe_experts_w4a4* experts,
+                                           const moe_router* router, void* y_dev, void* ws_dev, size_t ws_bytes,
+                                           void* stream);
+
+/* moe_w4a4_forward_profiled: moe_w4a4_forward that also records CUDA events
+ * between its phases on `stream` (phase_events: 6 cudaEvent_t passed as
+ * void*, NULL entries skipped): [0] before the first kernel, [1] after the
+ * router, [2] after the permutation and the quantisation of x, [3] after
+ * gate_up + GELU + the quantisation of h, [4] after down, [5] after the
+ * combine.  Results are identical to moe_w4a4_forward. */
+NVFP4MOE_API nvfp4_status moe_w4a4_forward_profiled(const void* x_dev, int32_t T, const moe_experts_w4a4* experts,
+                                                    const moe_router* router, void* y_dev, void* ws_dev,
+                                                    size_t ws_bytes, void* stream, void* const* phase_events);
+
+/* Byte offsets inside a W4A4 workspace of what a finished moe_w4a4_forward
+ * leaves behind.  Each expert's slots are padded to whole tiles of
+ * tile_tokens rows: expert e's tiles start at tile p_e = sum over e' < e of
+ * ceil(counts[e'] / tile_tokens), and its sorted slot offsets[e] + n sits at
+ * padded row p_e * tile_tokens + n (padding rows hold zero codes and scales).
+ *   ids, weights, counts, offsets, sorted_slot, slot_pos: as moe_forward_views
+ *   x_codes u8 [rows, H/2] and h_codes u8 [rows, I/2]: E2M1 codes per padded
+ *     row (element 2k in the low nibble of byte k)
+ *   x_scales, h_scales: per tile p and 64-element group g of the row, a
+ *     512-byte chunk at (p * (H/64 or I/64) + g) * 512; the E4M3 scale of
+ *     tile row r and block 4 g + i at byte 16 (r % 32) + 4 (r / 32) + i.
+ * tile_tokens is 16 for T <= 256, 64 for T <= 1024, else 128. */
+typedef struct {
+  size_t ids, weights, counts, offsets, sorted_slot, slot_pos;
+  size_t x_codes, x_scales, h_codes, h_scales;
+  int32_t tile_tokens, max_tiles;
+} moe_w4a4_views;
+NVFP4MOE_API nvfp4_status moe_w4a4_workspace_views(int32_t T, const moe_experts_w4a4* experts,
+                                                   const moe_router* router, moe_w4a4_views* out);
+
+/* ---------------------------------------------------------------------------
  * moe_permute: the token permutation of moe_nvfp4_forward on its own -- the
  * T*8 routing slots s = t*8 + j grouped by expert with a stable counting sort
  * (the sort-by-expert step of the batched expert kernel, "Gemma 4 26B-A4B

@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import importlib
 
-_API = {"MoeLayer", "MoeBlock", "DenseParts", "Aff4Experts", "Aff4Layer", "Router", "Experts", "quantize", "dequantize", "route", "permute", "residual_rmsnorm",
+_API = {"MoeLayer", "MoeBlock", "DenseParts", "Aff4Experts", "Aff4Layer", "W4A4Layer", "Router", "Experts", "quantize", "dequantize", "route", "permute", "residual_rmsnorm",
         "device_status", "forward_views", "unscaled_hidden"}
 _CAPI = {"NVFP4Error", "check", "status_string"}
 

@@ -265,6 +265,65 @@ class Aff4Layer:
         return self.workspace[v.ids:v.ids + T * TOP_K * 4].view(torch.int32).view(T, TOP_K)
 
 
+class W4A4Layer:
+    """One sparse MoE branch in the W4A4 form (moe_w4a4_forward): NVFP4
+    experts, their block scales packed once into the tensor core's order, the
+    static input globals gx (experts' input) and gh (hidden), and a workspace
+    for up to `max_tokens` tokens."""
+
+    def __init__(self, experts: Experts, router: Router, gx: float, gh: float, max_tokens: int, stream=None):
+        self.experts, self.router = experts, router
+        dev = experts.gate_up_q.device
+        ex = experts.c_struct()
+        E_ = experts.gate_up_q.shape[0]
+        self.gate_up_sf = torch.empty(capi.moe_w4a4_scale_bytes(E_, 0), dtype=torch.uint8, device=dev)
+        self.down_sf = torch.empty(capi.moe_w4a4_scale_bytes(E_, 1), dtype=torch.uint8, device=dev)
+        check(capi.moe_w4a4_pack_scales(ctypes.byref(ex), _ptr(self.gate_up_sf), _ptr(self.down_sf),
+                                        _stream(stream)), "moe_w4a4_pack_scales")
+        self._xs = capi.moe_experts_w4a4(ex, _ptr(self.gate_up_sf), _ptr(self.down_sf), float(gx), float(gh))
+        self._rs = router.c_struct()
+        self.max_tokens = int(max_tokens)
+        nbytes = capi.moe_w4a4_workspace_bytes(self.max_tokens, ctypes.byref(self._xs), ctypes.byref(self._rs))
+        if nbytes == 0:
+            raise ValueError("unsupported experts/router configuration")
+        self.workspace = _workspace(nbytes, dev)
+
+    def forward_into(self, x: torch.Tensor, y: torch.Tensor, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError(f"T={T} exceeds max_tokens={self.max_tokens}")
+        check(capi.moe_w4a4_forward(_ptr(x), T, ctypes.byref(self._xs), ctypes.byref(self._rs), _ptr(y),
+                                    _ptr(self.workspace), self.workspace.numel(), _stream(stream)),
+              "moe_w4a4_forward")
+        return y
+
+    def __call__(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        return self.forward_into(x, torch.empty_like(x), stream)
+
+    def views(self, T: int) -> dict:
+        """What the last forward of T tokens left in the workspace, as device
+        tensors (layouts of moe_w4a4_workspace_views)."""
+        v = capi.moe_w4a4_views()
+        check(capi.moe_w4a4_workspace_views(T, ctypes.byref(self._xs), ctypes.byref(self._rs), ctypes.byref(v)),
+              "moe_w4a4_workspace_views")
+        ws, S = self.workspace, T * TOP_K
+        nt, mt = v.tile_tokens, v.max_tiles
+
+        def i32(off, n):
+            return ws[off:off + 4 * n].view(torch.int32)
+        return {
+            "ids": i32(v.ids, S).view(T, TOP_K),
+            "weights": ws[v.weights:v.weights + 4 * S].view(torch.float32).view(T, TOP_K),
+            "counts": i32(v.counts, E), "offsets": i32(v.offsets, E + 1),
+            "sorted_slot": i32(v.sorted_slot, S), "slot_pos": i32(v.slot_pos, S),
+            "x_codes": ws[v.x_codes:v.x_codes + mt * nt * (H // 2)].view(mt * nt, H // 2),
+            "x_scales": ws[v.x_scales:v.x_scales + mt * (H // 64) * 512],
+            "h_codes": ws[v.h_codes:v.h_codes + mt * nt * (I // 2)].view(mt * nt, I // 2),
+            "h_scales": ws[v.h_scales:v.h_scales + mt * (I // 64) * 512],
+            "tile_tokens": nt, "max_tiles": mt,
+        }
+
+
 @dataclasses.dataclass
 class DenseParts:
     """The full block's bf16 tensors besides the experts and the router: the

@@ -66,10 +66,23 @@ class moe_block(ctypes.Structure):
                 ("post_ff_norm", c_void_p), ("layer_scalar", c_void_p), ("dense_I", c_int32), ("eps", c_float)]
 
 
+class moe_experts_w4a4(ctypes.Structure):
+    _fields_ = [("experts", moe_experts), ("gate_up_sf", c_void_p), ("down_sf", c_void_p),
+                ("input_scale_gate_up", c_float), ("input_scale_down", c_float)]
+
+
+class moe_w4a4_views(ctypes.Structure):
+    _fields_ = [("ids", c_size_t), ("weights", c_size_t), ("counts", c_size_t), ("offsets", c_size_t),
+                ("sorted_slot", c_size_t), ("slot_pos", c_size_t), ("x_codes", c_size_t),
+                ("x_scales", c_size_t), ("h_codes", c_size_t), ("h_scales", c_size_t),
+                ("tile_tokens", c_int32), ("max_tiles", c_int32)]
+
+
 _R = ctypes.POINTER(moe_router)
 _X = ctypes.POINTER(moe_experts)
 _B = ctypes.POINTER(moe_block)
 _A = ctypes.POINTER(moe_experts_aff4)
+_W = ctypes.POINTER(moe_experts_w4a4)
 
 # name -> (restype, argtypes), in the order of the header
 SIGNATURES = {
@@ -93,6 +106,13 @@ SIGNATURES = {
     "moe_forward_workspace_views": (c_int32, [c_int32, _X, _R, ctypes.POINTER(moe_forward_views)]),
     "moe_block_workspace_bytes": (c_size_t, [c_int32, _B]),
     "moe_block_forward": (c_int32, [c_void_p, c_int32, _B, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_w4a4_scale_bytes": (c_size_t, [c_int32, c_int32]),
+    "moe_w4a4_pack_scales": (c_int32, [_X, c_void_p, c_void_p, c_void_p]),
+    "moe_w4a4_workspace_bytes": (c_size_t, [c_int32, _W, _R]),
+    "moe_w4a4_forward": (c_int32, [c_void_p, c_int32, _W, _R, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_w4a4_forward_profiled": (c_int32, [c_void_p, c_int32, _W, _R, c_void_p, c_void_p, c_size_t, c_void_p,
+                                            ctypes.POINTER(c_void_p)]),
+    "moe_w4a4_workspace_views": (c_int32, [c_int32, _W, _R, ctypes.POINTER(moe_w4a4_views)]),
     "moe_permute_workspace_bytes": (c_size_t, [c_int32]),
     "moe_permute": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                               c_void_p]),

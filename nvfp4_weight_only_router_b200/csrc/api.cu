@@ -578,6 +578,196 @@ nvfp4_status moe_block_forward(const void* x, int32_t T, const moe_block* b, voi
   return cuda_status(launch_block_final(fa, s));
 }
 
+// ------------------------------------------------------------------- W4A4
+namespace {
+
+struct W4A4Layout {
+  Region meta, ids, wts, chunk_count, sorted, pos, aq, asf, hq, hsf, obuf;
+  int S = 0, nchunks = 0, nt = 16, max_tiles = 0;
+  size_t total = 0;
+};
+
+W4A4Layout w4a4_layout(int T) {
+  W4A4Layout L;
+  Alloc al;
+  L.S = T * kTopK;
+  L.nchunks = (L.S + 1023) / 1024;
+  L.nt = w4a4_tile_tokens(T);
+  // every expert's slots padded to whole tiles: at most one partial tile each
+  L.max_tiles = (L.S + L.nt - 1) / L.nt + kE;
+  const size_t rows = (size_t)L.max_tiles * L.nt;
+  L.meta = al.take(sizeof(int) * kMetaInts);
+  L.ids = al.take(sizeof(int) * T * kTopK);
+  L.wts = al.take(sizeof(float) * T * kTopK);
+  L.chunk_count = al.take(sizeof(int) * (size_t)L.nchunks * kE);
+  L.sorted = al.take(sizeof(int) * L.S);
+  L.pos = al.take(sizeof(int) * L.S);
+  L.aq = al.take(rows * (kH / 2));
+  L.asf = al.take((size_t)L.max_tiles * (kH / 64) * 512);
+  L.hq = al.take(rows * (kI / 2));
+  L.hsf = al.take((size_t)L.max_tiles * (kI / 64) * 512);
+  L.obuf = al.take(sizeof(float) * (size_t)L.S * kH);
+  L.total = al.cur;
+  return L;
+}
+
+nvfp4_status check_experts_w4a4(const moe_experts_w4a4* x) {
+  if (!x) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_experts(&x->experts);
+  if (st != NVFP4_OK) return st;
+  if (!x->gate_up_sf || !x->down_sf) return NVFP4_ERR_INVALID_ARG;
+  const float gs[2] = {x->input_scale_gate_up, x->input_scale_down};
+  for (float g : gs)
+    if (!(g > 0.f) || !std::isfinite(g)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(x->gate_up_sf, 16) || !aligned(x->down_sf, 16)) return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+size_t moe_w4a4_scale_bytes(int32_t E, int32_t which) {
+  if (E < 1 || E > (1 << 20)) return 0;
+  if (which == 0) return (size_t)E * (2 * kI) * (kH / kBlock);
+  if (which == 1) return (size_t)E * kH * (kI / kBlock);
+  return 0;
+}
+
+nvfp4_status moe_w4a4_pack_scales(const moe_experts* ex, uint8_t* gu_sf, uint8_t* dn_sf, void* stream) {
+  nvfp4_status st = check_experts(ex);
+  if (st != NVFP4_OK) return st;
+  if (!gu_sf || !dn_sf) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(gu_sf, 16) || !aligned(dn_sf, 16)) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = launch_w4a4_pack_scales(ex->gate_up_s, ex->E, 0, gu_sf, s);
+  if (e == cudaSuccess) e = launch_w4a4_pack_scales(ex->down_s, ex->E, 1, dn_sf, s);
+  return cuda_status(e);
+}
+
+size_t moe_w4a4_workspace_bytes(int32_t T, const moe_experts_w4a4* ex, const moe_router* r) {
+  if (T < 1 || T > 65536 || check_experts_w4a4(ex) != NVFP4_OK || check_router(r, true) != NVFP4_OK) return 0;
+  return w4a4_layout(T).total;
+}
+
+nvfp4_status moe_w4a4_workspace_views(int32_t T, const moe_experts_w4a4* ex, const moe_router* r,
+                                      moe_w4a4_views* out) {
+  if (!out || T < 1 || T > 65536) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_experts_w4a4(ex);
+  if (st == NVFP4_OK) st = check_router(r, true);
+  if (st != NVFP4_OK) return st;
+  const W4A4Layout L = w4a4_layout(T);
+  out->ids = L.ids.off;
+  out->weights = L.wts.off;
+  out->counts = L.meta.off + sizeof(int) * kMetaCounts;
+  out->offsets = L.meta.off + sizeof(int) * kMetaOffsets;
+  out->sorted_slot = L.sorted.off;
+  out->slot_pos = L.pos.off;
+  out->x_codes = L.aq.off;
+  out->x_scales = L.asf.off;
+  out->h_codes = L.hq.off;
+  out->h_scales = L.hsf.off;
+  out->tile_tokens = L.nt;
+  out->max_tiles = L.max_tiles;
+  return NVFP4_OK;
+}
+
+static nvfp4_status w4a4_forward_impl(const void* x, int32_t T, const moe_experts_w4a4* ex, const moe_router* r,
+                                      void* y, void* ws, size_t ws_bytes, void* stream, void* const* ev) {
+  if (T < 1 || T > 65536 || !x || !y) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_experts_w4a4(ex);
+  if (st == NVFP4_OK) st = check_router(r, true);
+  if (st != NVFP4_OK) return st;
+  if (!aligned(x, 16) || !aligned(y, 16)) return NVFP4_ERR_ALIGNMENT;
+  const W4A4Layout L = w4a4_layout(T);
+  if (!ws || ws_bytes < L.total) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = as_stream(stream);
+  int* status = device_status_ptr();
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (ev && cudaStreamIsCapturing(s, &cap) != cudaSuccess) return cuda_fail(cudaGetLastError());
+  auto mark = [&](int i) -> bool {
+    if (!ev || !ev[i]) return true;
+    cudaEvent_t evt = static_cast<cudaEvent_t>(ev[i]);
+    if (cap == cudaStreamCaptureStatusActive)
+      return cudaEventRecordWithFlags(evt, s, cudaEventRecordExternal) == cudaSuccess;
+    return cudaEventRecord(evt, s) == cudaSuccess;
+  };
+  if (!mark(0)) return cuda_fail(cudaGetLastError());
+  cudaError_t e = cudaMemsetAsync(at<int>(ws, L.meta), 0, L.meta.bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int32_t* ids = at<int32_t>(ws, L.ids);
+  float* wts = at<float>(ws, L.wts);
+  RouteArgs ra = make_route_args(x, T, r, ids, wts, status);
+  const bool fused_permute = ra.few_tokens && L.S <= kFusedPermuteMaxSlots;
+  PermuteArgs pa;
+  pa.ids = ids;
+  pa.S = L.S;
+  pa.nchunks = L.nchunks;
+  pa.meta = at<int>(ws, L.meta);
+  pa.chunk_count = at<int>(ws, L.chunk_count);
+  pa.sorted_slot = at<int>(ws, L.sorted);
+  pa.slot_pos = at<int>(ws, L.pos);
+  pa.status = status;
+  if (fused_permute) {
+    ra.meta = pa.meta;
+    ra.sorted_slot = pa.sorted_slot;
+    ra.slot_pos = pa.slot_pos;
+  }
+  if ((e = launch_route(ra, s)) != cudaSuccess || !mark(1)) return cuda_fail(e);
+  if (!fused_permute && (e = launch_permute(pa, s)) != cudaSuccess) return cuda_fail(e);
+
+  const moe_experts& w = ex->experts;
+  uint8_t* aq = at<uint8_t>(ws, L.aq);
+  uint8_t* asf = at<uint8_t>(ws, L.asf);
+  uint8_t* hq = at<uint8_t>(ws, L.hq);
+  uint8_t* hsf = at<uint8_t>(ws, L.hsf);
+  e = launch_w4a4_act_quant(static_cast<const uint16_t*>(x), pa.meta, pa.sorted_slot, T, kTopK,
+                            ex->input_scale_gate_up, L.nt, L.max_tiles, aq, asf, status, s);
+  if (e != cudaSuccess || !mark(2)) return cuda_fail(e);
+  W4A4Args ga;
+  ga.wq = w.gate_up_q;
+  ga.wsf = ex->gate_up_sf;
+  ga.wg = w.gate_up_g;
+  ga.gin = ex->input_scale_gate_up;
+  ga.gh = ex->input_scale_down;
+  ga.aq = aq;
+  ga.asf = asf;
+  ga.hq = hq;
+  ga.hsf = hsf;
+  ga.meta = pa.meta;
+  ga.sorted_slot = pa.sorted_slot;
+  ga.wts = wts;
+  ga.obuf = at<float>(ws, L.obuf);
+  ga.max_tiles = L.max_tiles;
+  ga.status = status;
+  if ((e = launch_w4a4_gemm(ga, 0, L.nt, s)) != cudaSuccess || !mark(3)) return cuda_fail(e);
+  W4A4Args da = ga;
+  da.wq = w.down_q;
+  da.wsf = ex->down_sf;
+  da.wg = w.down_g;
+  da.gin = ex->input_scale_down;
+  da.aq = hq;
+  da.asf = hsf;
+  if ((e = launch_w4a4_gemm(da, 1, L.nt, s)) != cudaSuccess || !mark(4)) return cuda_fail(e);
+  ExpertArgs xa{};
+  xa.T = T;
+  xa.spt = kTopK;
+  xa.slot_pos = pa.slot_pos;
+  xa.obuf = ga.obuf;
+  xa.y = y;
+  if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
+nvfp4_status moe_w4a4_forward(const void* x, int32_t T, const moe_experts_w4a4* ex, const moe_router* r, void* y,
+                              void* ws, size_t ws_bytes, void* stream) {
+  return w4a4_forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, nullptr);
+}
+
+nvfp4_status moe_w4a4_forward_profiled(const void* x, int32_t T, const moe_experts_w4a4* ex, const moe_router* r,
+                                       void* y, void* ws, size_t ws_bytes, void* stream, void* const* phase_events) {
+  return w4a4_forward_impl(x, T, ex, r, y, ws, ws_bytes, stream, phase_events);
+}
+
 nvfp4_status moe_nvfp4_forward(const void* x, int32_t T, const moe_experts* ex, const moe_router* r,
                                void* y, void* ws, size_t ws_bytes, void* stream) {
   const nvfp4_status st = check_experts(ex);

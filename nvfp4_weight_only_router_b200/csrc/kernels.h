@@ -108,6 +108,35 @@ cudaError_t launch_gather_sorted(const ExpertArgs& a, cudaStream_t st);
 cudaError_t launch_moe_gate_up(const ExpertArgs& a, int nt, cudaStream_t st);
 cudaError_t launch_moe_down(const ExpertArgs& a, int nt, cudaStream_t st);
 
+// W4A4 experts on the block-scaled FP4 tensor cores (w4a4.cu).
+// Tokens per tile for T tokens (16, 64 or 128).
+int w4a4_tile_tokens(int T);
+// Packed block scales of one projection (kind 0 gate_up, 1 down) of E experts.
+cudaError_t launch_w4a4_pack_scales(const uint8_t* s, int E, int kind, uint8_t* out, cudaStream_t st);
+// x rows of each expert's padded token tiles -> E2M1 codes aq [max_tiles*nt, H/2]
+// and scale chunks asf under the static global gx.
+cudaError_t launch_w4a4_act_quant(const uint16_t* x, const int* meta, const int* sorted_slot, int T, int spt, float gx,
+                                  int nt, int max_tiles, uint8_t* aq, uint8_t* asf, int* status, cudaStream_t st);
+struct W4A4Args {
+  const uint8_t* wq;        // weight codes of this GEMM [E*N, K/2]
+  const uint8_t* wsf;       // its packed scales
+  const float* wg;          // its FP32 globals [E]
+  float gin;                // global of its input (Gx for gate_up, Gh for down)
+  float gh;                 // gate_up: the global the hidden is quantised under
+  const uint8_t* aq;        // input codes [max_tiles*nt, K/2]
+  const uint8_t* asf;       // input scale chunks
+  uint8_t* hq;              // gate_up: hidden codes [max_tiles*nt, I/2]
+  uint8_t* hsf;             // gate_up: hidden scale chunks
+  const int* meta;
+  const int* sorted_slot;
+  const float* wts;         // routing weights per slot
+  float* obuf;              // down: per-slot rows [S, H] (x weight x G_d x Gh)
+  int max_tiles;
+  int* status;
+};
+// kind 0 gate_up (+ GELU gate + hidden quantisation), 1 down
+cudaError_t launch_w4a4_gemm(const W4A4Args& a, int kind, int nt, cudaStream_t st);
+
 // The full block's dense MLP GEMMs (bf16 x bf16 -> fp32 on tcgen05).
 //   gate_up: w0 = gate [2112, H], w1 = up [2112, H], b0 = X [T, H] (bf16);
 //            out [splits][T][2 * 2112]: gate rows 0..2111, then up rows

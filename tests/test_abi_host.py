@@ -25,7 +25,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported(capi):
     names = header_functions()
-    assert len(names) == 24
+    assert len(names) == 30
     for n in names:
         assert hasattr(capi.lib, n), n
         assert n in capi.SIGNATURES, n
@@ -217,3 +217,33 @@ def test_aff4_validation(capi):
     bad = c.moe_experts_aff4(4096, 4096 + 2, 4096, 4096, 4096, 4096, 128, 2816, 704)
     assert c.moe_aff4_forward(P, 1, ctypes.byref(bad), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_ALIGNMENT
     assert c.moe_aff4_forward(P, 1, ctypes.byref(a), ctypes.byref(r), P, P, 0, None) == c.NVFP4_ERR_WORKSPACE
+
+
+def _w4a4(c, gx=0.003, gh=0.0007, sf=4096):
+    return c.moe_experts_w4a4(_experts(c), sf, sf, gx, gh)
+
+
+def test_w4a4_validation(capi):
+    c = capi
+    r, w = _router(c), _w4a4(c)
+    assert c.moe_w4a4_scale_bytes(128, 0) == 128 * 1408 * 176
+    assert c.moe_w4a4_scale_bytes(128, 1) == 128 * 2816 * 44
+    assert c.moe_w4a4_scale_bytes(0, 0) == 0 and c.moe_w4a4_scale_bytes(128, 2) == 0
+    sizes = [c.moe_w4a4_workspace_bytes(T, ctypes.byref(w), ctypes.byref(r)) for T in (1, 64, 4096)]
+    assert 0 < sizes[0] < sizes[1] < sizes[2]
+    assert c.moe_w4a4_workspace_bytes(65537, ctypes.byref(w), ctypes.byref(r)) == 0
+    v = c.moe_w4a4_views()
+    assert c.moe_w4a4_workspace_views(64, ctypes.byref(w), ctypes.byref(r), ctypes.byref(v)) == c.NVFP4_OK
+    assert v.tile_tokens == 16 and v.max_tiles == 512 // 16 + 128
+    assert c.moe_w4a4_workspace_views(4096, ctypes.byref(w), ctypes.byref(r), ctypes.byref(v)) == c.NVFP4_OK
+    assert v.tile_tokens == 128 and v.max_tiles == 32768 // 128 + 128
+    P, n = 4096, sizes[0]
+    assert c.moe_w4a4_forward(P, 1, ctypes.byref(w), ctypes.byref(r), P, P, n - 1, None) == c.NVFP4_ERR_WORKSPACE
+    assert c.moe_w4a4_forward(None, 1, ctypes.byref(w), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_INVALID_ARG
+    for bad in (_w4a4(c, gx=0.0), _w4a4(c, gh=float("inf")), _w4a4(c, gx=float("nan")), _w4a4(c, sf=None)):
+        assert c.moe_w4a4_forward(P, 1, ctypes.byref(bad), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_w4a4_forward(P, 1, ctypes.byref(_w4a4(c, sf=4096 + 8)), ctypes.byref(r), P, P, n,
+                              None) == c.NVFP4_ERR_ALIGNMENT
+    x = _experts(c, I=512)
+    assert c.moe_w4a4_pack_scales(ctypes.byref(x), P, P, None) == c.NVFP4_ERR_UNSUPPORTED
+    assert c.moe_w4a4_pack_scales(ctypes.byref(_experts(c)), None, P, None) == c.NVFP4_ERR_INVALID_ARG

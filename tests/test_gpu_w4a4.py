@@ -1,0 +1,172 @@
+"""moe_w4a4_forward (NVFP4 activations on the block-scaled FP4 tensor cores)
+on the GPU against the W4A4 oracle.
+
+What is unique is compared exactly; where a floating-point sum decides an
+integer the comparison allows what that sum may legitimately decide:
+  * packed weight scales: bit-exact against the documented chunk layout;
+  * x codes and scales: bit-exact (both sides quantise the same bf16 values
+    with the same fp32 steps);
+  * hidden codes and scales: the GPU forms h from fp32 tensor-core sums, the
+    oracle from fp64 ones, so a block may round differently where h / d lies
+    at a rounding threshold to within the sums' difference; such blocks must
+    be rare and still a valid rounding of the oracle's h;
+  * y against the oracle's down GEMM and combine on the GPU's own hidden
+    codes: the forward bar (bf16 output, fp32 against fp64 sums);
+  * y end to end against the oracle: the forward bar widened by the few
+    hidden blocks that may round the other way.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as gen
+import nvfp4_weight_only_router_b200 as lib
+from oracle import formats as F
+from oracle import moe as M
+from oracle import w4a4 as W
+from tests.gpu_common import bf16_from_dev, bf16_to_dev, check_forward, check_ids, forward_errors
+
+pytestmark = pytest.mark.gpu
+
+H, I, E, K8 = 2816, 704, 128, 8
+GX, GH = gen.W4A4_GX, gen.W4A4_GH
+
+
+@pytest.fixture(scope="module")
+def layer(layer0, dev):
+    return lib.W4A4Layer(layer0["dex"], layer0["drt"], GX, GH, max_tokens=4096)
+
+
+def _padded_rows(counts, offsets, nt):
+    """Padded row of every sorted position (the documented layout)."""
+    tiles = (counts + nt - 1) // nt
+    start = np.concatenate([[0], np.cumsum(tiles)[:-1]]) * nt
+    rows = np.empty(int(offsets[-1]), np.int64)
+    for e in range(E):
+        rows[offsets[e]:offsets[e + 1]] = start[e] + np.arange(counts[e])
+    return rows
+
+
+def _chunk_scales(chunks, rows, nt, K):
+    """Scales [len(rows), K/16] of the given padded rows from the 512-byte chunks."""
+    g = K // 64
+    tile, r = rows // nt, rows % nt
+    b = np.arange(K // 16)
+    idx = (tile[:, None] * g + b[None, :] // 4) * 512 + 16 * (r[:, None] % 32) + 4 * (r[:, None] // 32) + b[None, :] % 4
+    return chunks[idx]
+
+
+def test_pack_scales_layout(layer, layer0):
+    """Chunk (e, j, q): byte 16 r0 + 4 r1 + i = scale of tile row r0 + 32 r1,
+    block 4 q + i; gate_up tile rows interleave the gate and up rows of 16
+    hidden units per lane quarter."""
+    ex = layer0["ex"]
+    gu = layer.gate_up_sf.cpu().numpy().reshape(E, 11, 44, 32, 4, 4)   # e, j, q, r0, r1, i
+    dn = layer.down_sf.cpu().numpy().reshape(E, 22, 11, 32, 4, 4)
+    L = np.arange(128).reshape(4, 32).T           # [r0, r1] -> tile row
+    qd, w = L >> 5, L & 31
+    for e in (0, 77, 127):
+        for j in (0, 5, 10):
+            grow = np.where(w < 16, 0, I) + j * 64 + qd * 16 + (w & 15)
+            want = ex.gate_up_s[e][grow]                      # [32, 4, 176]
+            want = want.reshape(32, 4, 44, 4).transpose(2, 0, 1, 3)
+            assert np.array_equal(gu[e, j], want)
+        for j in (0, 13, 21):
+            want = ex.down_s[e][j * 128 + L].reshape(32, 4, 11, 4).transpose(2, 0, 1, 3)
+            assert np.array_equal(dn[e, j], want)
+
+
+def _run(layer, dev, x):
+    T = x.shape[0]
+    y = layer(bf16_to_dev(x, dev))
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0
+    v = {k: (t.cpu().numpy() if isinstance(t, torch.Tensor) else t) for k, t in layer.views(T).items()}
+    return bf16_from_dev(y), v
+
+
+def _check_valid_rounding(codes, scales, h):
+    """Blocks [n, 16] whose codes and scale the GPU chose differently from the
+    oracle: each must be the method's rounding of some h' within the fp32
+    sums' error of the oracle's h (relative 1e-5 of the element plus 1e-6 of
+    the block maximum).  Both roundings are monotone, so the GPU's scale must
+    lie between those of the block maxima at the ends of that range, and each
+    code, under the GPU's scale, between the codes of the element's ends."""
+    tol = 1e-5 * np.abs(h) + 1e-6 * np.abs(h).max(axis=1, keepdims=True)
+    amax = np.abs(h).max(axis=1)
+    tmax = tol.max(axis=1)
+    f32 = np.float32
+    s_lo = F.e4m3_encode_satfinite(((f32(np.maximum(amax - tmax, 0)) / f32(6)) / GH).astype(np.float64))
+    s_hi = F.e4m3_encode_satfinite(((f32(amax + tmax) / f32(6)) / GH).astype(np.float64))
+    assert np.all((s_lo <= scales) & (scales <= s_hi)), "hidden block scale outside its rounding range"
+    d = (F.e4m3_decode(scales).astype(f32) * GH).astype(f32)[:, None]
+    v_lo = F.e2m1_decode(F.e2m1_encode((h - tol).astype(f32) / d))
+    v_hi = F.e2m1_decode(F.e2m1_encode((h + tol).astype(f32) / d))
+    v = F.e2m1_decode(codes)
+    assert np.all((v_lo <= v) & (v <= v_hi)), "hidden code outside its rounding range"
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 300, 2048])
+def test_w4a4_forward(layer, layer0, dev, T):
+    """T <= 256: 16-token tiles; 300: 64; 2048: 128 (the oracle on 12 sampled
+    tokens above 64)."""
+    ex, rt = layer0["ex"], layer0["rt"]
+    x = gen.make_x(900 + T, T)
+    y, v = _run(layer, dev, x)
+    nt = v["tile_tokens"]
+    rows_of_pos = _padded_rows(v["counts"].astype(np.int64), v["offsets"].astype(np.int64), nt)
+    toks = np.arange(T) if T <= 64 else np.unique(np.r_[0, T - 1, np.random.default_rng(T).choice(T, 10, replace=False)])
+    ids0, _, logits = M.route(x[toks], rt)
+    differ = check_ids(v["ids"][toks], ids0, logits)
+    override = np.where(differ[:, None], v["ids"][toks], ids0) if differ.any() else None
+    ref = W.forward(x[toks], ex, rt, GX, GH, ids_override=override, return_parts=True)
+
+    # x codes and scales: every slot of a sampled token holds its token's quantised row
+    slots = (toks[:, None] * K8 + np.arange(K8)[None, :]).ravel()
+    prow = rows_of_pos[v["slot_pos"][slots]]
+    xq = np.repeat(ref["xq"], K8, axis=0)
+    xs = np.repeat(ref["xs"], K8, axis=0)
+    assert np.array_equal(v["x_codes"][prow], xq)
+    assert np.array_equal(_chunk_scales(v["x_scales"], prow, nt, H), xs)
+
+    # hidden codes: rare, valid threshold decisions only
+    hq_gpu = v["h_codes"][prow]
+    hs_gpu = _chunk_scales(v["h_scales"], prow, nt, I)
+    local = (np.arange(len(toks))[:, None] * K8 + np.arange(K8)[None, :]).ravel()
+    hq_ref, hs_ref, h32 = ref["hq"][local], ref["hs"][local], ref["h32"][local]
+    codes_gpu, codes_ref = F.unpack_nibbles(hq_gpu), F.unpack_nibbles(hq_ref)
+    bad = (codes_gpu != codes_ref).reshape(len(local), I // 16, 16).any(-1) | (hs_gpu != hs_ref)
+    assert bad.mean() < 2e-3, f"{bad.mean():.2e} of hidden blocks differ"
+    if bad.any():
+        _check_valid_rounding(codes_gpu.reshape(len(local), I // 16, 16)[bad], hs_gpu[bad],
+                              h32.astype(np.float64).reshape(len(local), I // 16, 16)[bad])
+
+    # y from the GPU's own hidden codes: the forward bar
+    y_own = W.down_from_codes(hq_gpu, hs_gpu, GH, ref["ids"], ref["w"], ex, len(toks))
+    check_forward(y[toks], y_own)
+    # end to end
+    rel, mx = forward_errors(y[toks], ref["y64"])
+    assert rel <= 4e-3 and mx <= 4e-2, (rel, mx)
+
+
+def test_w4a4_padding_rows_are_zero(layer, dev):
+    T = 24
+    x = gen.make_x(950, T)
+    _, v = _run(layer, dev, x)
+    nt = v["tile_tokens"]
+    counts = v["counts"].astype(np.int64)
+    rows = _padded_rows(counts, v["offsets"].astype(np.int64), nt)
+    total = int(((counts + nt - 1) // nt).sum()) * nt
+    pad = np.setdiff1d(np.arange(total), rows)
+    assert pad.size > 0
+    assert not v["x_codes"][pad].any() and not v["h_codes"][pad].any()
+    assert not _chunk_scales(v["x_scales"], pad, nt, H).any()
+    assert not _chunk_scales(v["h_scales"], pad, nt, I).any()
+
+
+def test_w4a4_repeat_is_deterministic(layer, dev):
+    x = bf16_to_dev(gen.make_x(960, 512), dev)
+    y1 = layer(x)
+    y2 = layer(x)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
