@@ -340,31 +340,36 @@ NVFP4MOE_API nvfp4_status moe_block_forward(const void* x_dev, int32_t T, const 
  * multiplies those codes with the down weights', o = w G_d Gh acc per slot,
  * and y[t] = bf16(sum over the token's 8 slots in slot order).
  *
- * The weights are those of moe_experts, plus their block scales copied once
- * into the order the tensor core reads them (moe_w4a4_pack_scales): per
- * expert, per 128-row tile of the projection and per 64 elements of K, one
- * 512-byte chunk.
+ * The weights are those of moe_experts, copied once into the tensor core's
+ * order by moe_w4a4_pack, so that every pipeline stage reads one contiguous
+ * block: per expert, per 128-row tile of the projection (gate_up tiles hold
+ * the gate rows of 16 hidden units then their 16 up rows, four times) and
+ * per 256 elements of K, the tile's codes as 128 rows of 128 bytes in the
+ * 128-byte swizzle (16-byte piece p of row r stored at piece p ^ (r % 8));
+ * and per 64 elements of K, the tile's block scales as one 512-byte chunk
+ * (row r = r0 + 32 r1 at byte 16 r0 + 4 r1).
  * ------------------------------------------------------------------------- */
 typedef struct {
   moe_experts experts;           /* codes, block scales and globals (moe_nvfp4_forward's) */
-  const uint8_t* gate_up_sf;     /* moe_w4a4_scale_bytes(E, 0) bytes from moe_w4a4_pack_scales */
-  const uint8_t* down_sf;        /* moe_w4a4_scale_bytes(E, 1) bytes */
+  const uint8_t* gate_up_pk;     /* moe_w4a4_pack_bytes(E, 0) bytes from moe_w4a4_pack */
+  const uint8_t* down_pk;        /* moe_w4a4_pack_bytes(E, 1) bytes */
+  const uint8_t* gate_up_sf;     /* moe_w4a4_pack_bytes(E, 2) bytes */
+  const uint8_t* down_sf;        /* moe_w4a4_pack_bytes(E, 3) bytes */
   float input_scale_gate_up;     /* Gx > 0, finite */
   float input_scale_down;        /* Gh > 0, finite */
 } moe_experts_w4a4;
 
-/* Bytes of the packed block scales of the gate_up (which = 0) or down
- * (which = 1) projections of E experts: E * N * K / 16 (0 for E < 1 or another
- * `which`). */
-NVFP4MOE_API size_t moe_w4a4_scale_bytes(int32_t E, int32_t which);
+/* Bytes of the packed gate_up codes (which = 0), down codes (1), gate_up
+ * block scales (2) or down block scales (3) of E experts (0 for E < 1 or
+ * another `which`). */
+NVFP4MOE_API size_t moe_w4a4_pack_bytes(int32_t E, int32_t which);
 
-/* moe_w4a4_pack_scales: copies experts->gate_up_s and down_s into the tensor
- * core's order, gate_up_sf_dev / down_sf_dev of moe_w4a4_scale_bytes(E, 0/1)
- * bytes (device, 16-byte aligned, caller-owned).  Run once per set of
- * weights; asynchronous on `stream`.  Same shape requirements as
- * moe_nvfp4_forward. */
-NVFP4MOE_API nvfp4_status moe_w4a4_pack_scales(const moe_experts* experts, uint8_t* gate_up_sf_dev,
-                                               uint8_t* down_sf_dev, void* stream);
+/* moe_w4a4_pack: writes the four packed copies of `experts` (device buffers of
+ * moe_w4a4_pack_bytes(E, 0..3) bytes, 16-byte aligned, caller-owned).  Run
+ * once per set of weights; asynchronous on `stream`.  Same shape requirements
+ * as moe_nvfp4_forward. */
+NVFP4MOE_API nvfp4_status moe_w4a4_pack(const moe_experts* experts, uint8_t* gate_up_pk_dev, uint8_t* down_pk_dev,
+                                        uint8_t* gate_up_sf_dev, uint8_t* down_sf_dev, void* stream);
 
 /* moe_w4a4_forward: y_dev bf16 [T, H] from x_dev bf16 [T, H] as described
  * above; 1 <= T <= 65536, router and experts as for moe_nvfp4_forward.
@@ -388,11 +393,15 @@ NVFP4MOE_API nvfp4_status moe_w4a4_forward_profiled(const void* x_dev, int32_t T
 /* Byte offsets inside a W4A4 workspace of what a finished moe_w4a4_forward
  * leaves behind.  Each expert's slots are padded to whole tiles of
  * tile_tokens rows: expert e's tiles start at tile p_e = sum over e' < e of
- * ceil(counts[e'] / tile_tokens), and its sorted slot offsets[e] + n sits at
- * padded row p_e * tile_tokens + n (padding rows hold zero codes and scales).
+ * ceil(counts[e'] / tile_tokens), and its sorted slot offsets[e] + n is row
+ * n' = (n mod tile_tokens) of tile p_e + n / tile_tokens.  Padding rows of x
+ * are unspecified; those of h hold zero codes and scales.
  *   ids, weights, counts, offsets, sorted_slot, slot_pos: as moe_forward_views
- *   x_codes u8 [rows, H/2] and h_codes u8 [rows, I/2]: E2M1 codes per padded
- *     row (element 2k in the low nibble of byte k)
+ *   x_codes, h_codes: E2M1 codes (element 2k in the low nibble of byte k) per
+ *     tile p and 256-element K chunk c, a block of tile_tokens rows of 128
+ *     bytes at (p * C + c) * tile_tokens * 128 (C = 11 for x, 3 for h, whose
+ *     rows end at byte 352 of 384), row r's byte k of the chunk at
+ *     128 r + 16 ((k / 16) ^ (r % 8)) + k % 16
  *   x_scales, h_scales: per tile p and 64-element group g of the row, a
  *     512-byte chunk at (p * (H/64 or I/64) + g) * 512; the E4M3 scale of
  *     tile row r and block 4 g + i at byte 16 (r % 32) + 4 (r / 32) + i.

@@ -276,11 +276,12 @@ class W4A4Layer:
         dev = experts.gate_up_q.device
         ex = experts.c_struct()
         E_ = experts.gate_up_q.shape[0]
-        self.gate_up_sf = torch.empty(capi.moe_w4a4_scale_bytes(E_, 0), dtype=torch.uint8, device=dev)
-        self.down_sf = torch.empty(capi.moe_w4a4_scale_bytes(E_, 1), dtype=torch.uint8, device=dev)
-        check(capi.moe_w4a4_pack_scales(ctypes.byref(ex), _ptr(self.gate_up_sf), _ptr(self.down_sf),
-                                        _stream(stream)), "moe_w4a4_pack_scales")
-        self._xs = capi.moe_experts_w4a4(ex, _ptr(self.gate_up_sf), _ptr(self.down_sf), float(gx), float(gh))
+        self.gate_up_pk, self.down_pk, self.gate_up_sf, self.down_sf = (
+            torch.empty(capi.moe_w4a4_pack_bytes(E_, w), dtype=torch.uint8, device=dev) for w in range(4))
+        check(capi.moe_w4a4_pack(ctypes.byref(ex), _ptr(self.gate_up_pk), _ptr(self.down_pk), _ptr(self.gate_up_sf),
+                                 _ptr(self.down_sf), _stream(stream)), "moe_w4a4_pack")
+        self._xs = capi.moe_experts_w4a4(ex, _ptr(self.gate_up_pk), _ptr(self.down_pk), _ptr(self.gate_up_sf),
+                                         _ptr(self.down_sf), float(gx), float(gh))
         self._rs = router.c_struct()
         self.max_tokens = int(max_tokens)
         nbytes = capi.moe_w4a4_workspace_bytes(self.max_tokens, ctypes.byref(self._xs), ctypes.byref(self._rs))
@@ -316,9 +317,9 @@ class W4A4Layer:
             "weights": ws[v.weights:v.weights + 4 * S].view(torch.float32).view(T, TOP_K),
             "counts": i32(v.counts, E), "offsets": i32(v.offsets, E + 1),
             "sorted_slot": i32(v.sorted_slot, S), "slot_pos": i32(v.slot_pos, S),
-            "x_codes": ws[v.x_codes:v.x_codes + mt * nt * (H // 2)].view(mt * nt, H // 2),
+            "x_codes": ws[v.x_codes:v.x_codes + mt * 11 * nt * 128],
             "x_scales": ws[v.x_scales:v.x_scales + mt * (H // 64) * 512],
-            "h_codes": ws[v.h_codes:v.h_codes + mt * nt * (I // 2)].view(mt * nt, I // 2),
+            "h_codes": ws[v.h_codes:v.h_codes + mt * 3 * nt * 128],
             "h_scales": ws[v.h_scales:v.h_scales + mt * (I // 64) * 512],
             "tile_tokens": nt, "max_tiles": mt,
         }

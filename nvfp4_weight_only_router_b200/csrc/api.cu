@@ -582,7 +582,7 @@ nvfp4_status moe_block_forward(const void* x, int32_t T, const moe_block* b, voi
 namespace {
 
 struct W4A4Layout {
-  Region meta, ids, wts, chunk_count, sorted, pos, aq, asf, hq, hsf, obuf;
+  Region meta, ids, wts, chunk_count, sorted, pos, aq, asf, roww, hq, hsf, obuf;
   int S = 0, nchunks = 0, nt = 16, max_tiles = 0;
   size_t total = 0;
 };
@@ -604,7 +604,8 @@ W4A4Layout w4a4_layout(int T) {
   L.pos = al.take(sizeof(int) * L.S);
   L.aq = al.take(rows * (kH / 2));
   L.asf = al.take((size_t)L.max_tiles * (kH / 64) * 512);
-  L.hq = al.take(rows * (kI / 2));
+  L.roww = al.take(sizeof(float) * rows);
+  L.hq = al.take(rows * 384);  // 3 chunks of 128 bytes per row
   L.hsf = al.take((size_t)L.max_tiles * (kI / 64) * 512);
   L.obuf = al.take(sizeof(float) * (size_t)L.S * kH);
   L.total = al.cur;
@@ -615,30 +616,40 @@ nvfp4_status check_experts_w4a4(const moe_experts_w4a4* x) {
   if (!x) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_experts(&x->experts);
   if (st != NVFP4_OK) return st;
-  if (!x->gate_up_sf || !x->down_sf) return NVFP4_ERR_INVALID_ARG;
+  if (!x->gate_up_pk || !x->down_pk || !x->gate_up_sf || !x->down_sf) return NVFP4_ERR_INVALID_ARG;
   const float gs[2] = {x->input_scale_gate_up, x->input_scale_down};
   for (float g : gs)
     if (!(g > 0.f) || !std::isfinite(g)) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(x->gate_up_sf, 16) || !aligned(x->down_sf, 16)) return NVFP4_ERR_ALIGNMENT;
+  const void* ps[] = {x->gate_up_pk, x->down_pk, x->gate_up_sf, x->down_sf};
+  for (const void* p : ps)
+    if (!aligned(p, 16)) return NVFP4_ERR_ALIGNMENT;
   return NVFP4_OK;
 }
 
 }  // namespace
 
-size_t moe_w4a4_scale_bytes(int32_t E, int32_t which) {
+size_t moe_w4a4_pack_bytes(int32_t E, int32_t which) {
   if (E < 1 || E > (1 << 20)) return 0;
-  if (which == 0) return (size_t)E * (2 * kI) * (kH / kBlock);
-  if (which == 1) return (size_t)E * kH * (kI / kBlock);
+  switch (which) {
+    case 0: return w4a4_packed_code_bytes(E, 0);
+    case 1: return w4a4_packed_code_bytes(E, 1);
+    case 2: return (size_t)E * (2 * kI) * (kH / kBlock);
+    case 3: return (size_t)E * kH * (kI / kBlock);
+  }
   return 0;
 }
 
-nvfp4_status moe_w4a4_pack_scales(const moe_experts* ex, uint8_t* gu_sf, uint8_t* dn_sf, void* stream) {
+nvfp4_status moe_w4a4_pack(const moe_experts* ex, uint8_t* gu_pk, uint8_t* dn_pk, uint8_t* gu_sf, uint8_t* dn_sf,
+                           void* stream) {
   nvfp4_status st = check_experts(ex);
   if (st != NVFP4_OK) return st;
-  if (!gu_sf || !dn_sf) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(gu_sf, 16) || !aligned(dn_sf, 16)) return NVFP4_ERR_ALIGNMENT;
+  if (!gu_pk || !dn_pk || !gu_sf || !dn_sf) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(gu_pk, 16) || !aligned(dn_pk, 16) || !aligned(gu_sf, 16) || !aligned(dn_sf, 16))
+    return NVFP4_ERR_ALIGNMENT;
   cudaStream_t s = as_stream(stream);
-  cudaError_t e = launch_w4a4_pack_scales(ex->gate_up_s, ex->E, 0, gu_sf, s);
+  cudaError_t e = launch_w4a4_pack_codes(ex->gate_up_q, ex->E, 0, gu_pk, s);
+  if (e == cudaSuccess) e = launch_w4a4_pack_codes(ex->down_q, ex->E, 1, dn_pk, s);
+  if (e == cudaSuccess) e = launch_w4a4_pack_scales(ex->gate_up_s, ex->E, 0, gu_sf, s);
   if (e == cudaSuccess) e = launch_w4a4_pack_scales(ex->down_s, ex->E, 1, dn_sf, s);
   return cuda_status(e);
 }
@@ -720,11 +731,12 @@ static nvfp4_status w4a4_forward_impl(const void* x, int32_t T, const moe_expert
   uint8_t* asf = at<uint8_t>(ws, L.asf);
   uint8_t* hq = at<uint8_t>(ws, L.hq);
   uint8_t* hsf = at<uint8_t>(ws, L.hsf);
-  e = launch_w4a4_act_quant(static_cast<const uint16_t*>(x), pa.meta, pa.sorted_slot, T, kTopK,
-                            ex->input_scale_gate_up, L.nt, L.max_tiles, aq, asf, status, s);
+  float* roww = at<float>(ws, L.roww);
+  e = launch_w4a4_act_quant(static_cast<const uint16_t*>(x), pa.meta, pa.slot_pos, wts, T, ex->input_scale_gate_up,
+                            L.nt, aq, asf, roww, status, s);
   if (e != cudaSuccess || !mark(2)) return cuda_fail(e);
   W4A4Args ga;
-  ga.wq = w.gate_up_q;
+  ga.wq = ex->gate_up_pk;
   ga.wsf = ex->gate_up_sf;
   ga.wg = w.gate_up_g;
   ga.gin = ex->input_scale_gate_up;
@@ -734,14 +746,13 @@ static nvfp4_status w4a4_forward_impl(const void* x, int32_t T, const moe_expert
   ga.hq = hq;
   ga.hsf = hsf;
   ga.meta = pa.meta;
-  ga.sorted_slot = pa.sorted_slot;
-  ga.wts = wts;
+  ga.roww = roww;
   ga.obuf = at<float>(ws, L.obuf);
   ga.max_tiles = L.max_tiles;
   ga.status = status;
   if ((e = launch_w4a4_gemm(ga, 0, L.nt, s)) != cudaSuccess || !mark(3)) return cuda_fail(e);
   W4A4Args da = ga;
-  da.wq = w.down_q;
+  da.wq = ex->down_pk;
   da.wsf = ex->down_sf;
   da.wg = w.down_g;
   da.gin = ex->input_scale_down;

@@ -111,25 +111,29 @@ cudaError_t launch_moe_down(const ExpertArgs& a, int nt, cudaStream_t st);
 // W4A4 experts on the block-scaled FP4 tensor cores (w4a4.cu).
 // Tokens per tile for T tokens (16, 64 or 128).
 int w4a4_tile_tokens(int T);
-// Packed block scales of one projection (kind 0 gate_up, 1 down) of E experts.
+// Packed block scales / codes of one projection (kind 0 gate_up, 1 down) of E experts.
 cudaError_t launch_w4a4_pack_scales(const uint8_t* s, int E, int kind, uint8_t* out, cudaStream_t st);
-// x rows of each expert's padded token tiles -> E2M1 codes aq [max_tiles*nt, H/2]
-// and scale chunks asf under the static global gx.
-cudaError_t launch_w4a4_act_quant(const uint16_t* x, const int* meta, const int* sorted_slot, int T, int spt, float gx,
-                                  int nt, int max_tiles, uint8_t* aq, uint8_t* asf, int* status, cudaStream_t st);
+cudaError_t launch_w4a4_pack_codes(const uint8_t* q, int E, int kind, uint8_t* out, cudaStream_t st);
+// Bytes of the packed codes of one projection (kind 0 gate_up, 1 down) of E experts.
+size_t w4a4_packed_code_bytes(int E, int kind);
+// Each token's x -> E2M1 codes aq (tile-major, 128-byte swizzled) and scale
+// chunks asf (static global gx) at the padded rows of its 8 slots, and each
+// slot's routing weight at its padded row of roww [max_tiles*nt].
+cudaError_t launch_w4a4_act_quant(const uint16_t* x, const int* meta, const int* slot_pos, const float* wts, int T,
+                                  float gx, int nt, uint8_t* aq, uint8_t* asf, float* roww, int* status,
+                                  cudaStream_t st);
 struct W4A4Args {
-  const uint8_t* wq;        // weight codes of this GEMM [E*N, K/2]
+  const uint8_t* wq;        // packed weight codes of this GEMM
   const uint8_t* wsf;       // its packed scales
   const float* wg;          // its FP32 globals [E]
   float gin;                // global of its input (Gx for gate_up, Gh for down)
   float gh;                 // gate_up: the global the hidden is quantised under
-  const uint8_t* aq;        // input codes [max_tiles*nt, K/2]
+  const uint8_t* aq;        // input codes, tile-major [max_tiles][K/256][nt][128 B]
   const uint8_t* asf;       // input scale chunks
-  uint8_t* hq;              // gate_up: hidden codes [max_tiles*nt, I/2]
+  uint8_t* hq;              // gate_up: hidden codes, tile-major [max_tiles][3][nt][128 B]
   uint8_t* hsf;             // gate_up: hidden scale chunks
   const int* meta;
-  const int* sorted_slot;
-  const float* wts;         // routing weights per slot
+  const float* roww;        // routing weight per padded row (0 for padding)
   float* obuf;              // down: per-slot rows [S, H] (x weight x G_d x Gh)
   int max_tiles;
   int* status;

@@ -13,11 +13,16 @@
 //             quantised per 16 hidden units under the static global Gh;
 //   down:     o[slot, r] = w_slot G_d Gh sum_k deq(h)[k] deq(W_d)[r, k].
 //
-// Layouts.  Each expert's tokens are padded to whole tiles of NT rows, so a
-// token tile is a plain TMA box and owns its scale chunks:
-//   activation codes  [tiles * NT, K/2]   (row = padded position)
-//   activation scales [tiles][K/64][512]  one 512-byte chunk per MMA K step
-//   weight scales     [E][N/128][K/64][512]  (moe_w4a4_pack_scales)
+// Layouts.  Every operand stage is one contiguous block that a single bulk
+// copy brings into shared memory in the form the MMA reads (K-major rows of
+// 128 bytes = 256 codes, 8-row atoms of 1024 bytes with the 16-byte piece
+// index XOR-ed with the row index: the 128-byte swizzle), so the weight
+// stream reads whole 16 KB blocks of HBM.  Each expert's tokens are padded to
+// whole tiles of NT rows:
+//   weight codes      [E][N/128][K/256][128 rows][128 B]   (moe_w4a4_pack)
+//   weight scales     [E][N/128][K/64][512]                (moe_w4a4_pack)
+//   activation codes  [tiles][K/256][NT rows][128 B]
+//   activation scales [tiles][K/64][512]
 // A 512-byte chunk holds the 4 scales of one K step for 128 rows, row
 // r = r0 + 32 r1 at byte 16 r0 + 4 r1 + (k / 16): the order in which one
 // tcgen05.cp (32 x 128 bit, copied to all four lane quarters) leaves them
@@ -25,8 +30,8 @@
 //
 // Tiles and warps as in the W4A16 tensor-core kernel: work tile = (expert,
 // token tile, 128 weight rows), K in 128-byte chunks (4 MMA K steps); warp 0
-// issues the TMA boxes and bulk copies, warp 1 the scale copies and MMAs (one
-// elected lane), warps 4-7 the epilogue.  A gate_up tile holds 64 hidden
+// issues the bulk copies, warp 2 the copies of the block scales into tensor
+// memory, warp 1 the MMAs (one elected lane), warps 4-7 the epilogue.  A gate_up tile holds 64 hidden
 // units: lane quarter q has gate rows of units 16q.. in lanes 0-15 and the
 // matching up rows in lanes 16-31.  Every wait is bounded.
 #include <algorithm>
@@ -41,9 +46,7 @@ namespace {
 
 constexpr int kF4Rows = 128;    // weight rows per tile (MMA M)
 constexpr int kSfChunk = 512;   // one MMA K step's block scales for 128 rows
-constexpr int kF4Warps = 8;
-constexpr int kF4Threads = kF4Warps * 32;
-constexpr int kF4Prod = 0, kF4Mma = 1, kF4Epi0 = 4;
+constexpr int kF4Prod = 0, kF4Mma = 1, kF4Sf = 2, kF4Epi0 = 4;
 constexpr int kF4TmemCols = 512;
 
 template <int KIND>
@@ -63,7 +66,12 @@ struct F4Cfg {
   static constexpr int B_BYTES = NT * 128;
   static constexpr int SF_BYTES = 4 * kSfChunk;                // 4 K steps per chunk
   static constexpr int STAGE = A_BYTES + B_BYTES + 2 * SF_BYTES;
-  static constexpr int STG = KIND == 0 ? NT * 16 : 1;          // epilogue staging floats per warp
+  // epilogue: NEPI sets of 4 warps (one per tensor-memory lane quarter), set
+  // h taking token columns [h TPS, (h + 1) TPS) of each tile
+  static constexpr int NEPI = NT >= 64 ? 2 : 1;
+  static constexpr int TPS = NT / NEPI;
+  static constexpr int THREADS = 32 * (kF4Epi0 + 4 * NEPI);
+  static constexpr int STG = KIND == 0 ? TPS * 16 : 1;         // epilogue staging floats per warp
   static constexpr int NS_SMEM = (224 * 1024 - 4 * 4 * STG) / STAGE;
   static constexpr int NS_TMEM = (kF4TmemCols - 2 * NT) / 32;  // 32 scale columns per stage
   static constexpr int NS_MIN = NS_SMEM < NS_TMEM ? NS_SMEM : NS_TMEM;
@@ -79,11 +87,12 @@ struct alignas(1024) F4Smem {
   uint8_t b[C::NS][C::B_BYTES];     // activation codes, NT rows x 128 bytes, 128B-swizzled
   uint8_t sfa[C::NS][C::SF_BYTES];  // weight scale chunks
   uint8_t sfb[C::NS][C::SF_BYTES];  // activation scale chunks
-  float stage[4][C::STG];           // gate_up: per epilogue warp, h[token][16 units]
-  float tokw[4][NT];                // down: per token column w_slot G_d Gh
-  uint64_t full[C::NS], empty[C::NS];
+  float stage[4 * C::NEPI][C::STG];  // gate_up: per epilogue warp, h[token][16 units]
+  // full[s]: the stage's copies landed; sf_ready[s]: its scales are in tensor
+  // memory; empty[s]: its MMAs completed (stage and scale columns free)
+  uint64_t full[C::NS], sf_ready[C::NS], empty[C::NS];
   uint64_t d_full[2], d_empty[2];
-  uint64_t fin;
+  uint64_t fin, sf_fin;
   uint32_t taddr;
   int mt_prefix[kE + 1];
   int abort_flag;
@@ -153,6 +162,12 @@ __device__ __forceinline__ int f4_tile_row(int e, int j, int L) {
   return e * kH + j * kF4Rows + L;
 }
 
+// Byte offset of byte k (0..127) of row r inside a block of 128-byte rows
+// stored in the 128-byte swizzle (16-byte piece index XOR row % 8).
+__host__ __device__ __forceinline__ uint32_t sw128(int r, int k) {
+  return (uint32_t)r * 128u + ((uint32_t)(((k >> 4) ^ r) & 7) << 4) + (uint32_t)(k & 15);
+}
+
 // Exclusive prefix over experts of their token tiles (ceil(count / nt)) into
 // prefix[0..E]; run by one full warp.
 __device__ __forceinline__ void tile_prefix_warp(const int* meta, int nt, int* prefix) {
@@ -190,6 +205,29 @@ __device__ __forceinline__ int expert_of_tile(const int* prefix, int tile) {
   return lo;
 }
 
+// ------------------------------------------------------------- code packing
+// out[(((e NJ + j) KCH + c) 128 + L) 128 + swizzled piece] = 16 bytes of
+// K bytes 128 c.. of weight row row(e, j, L) (zero past the row's end); one
+// 16-byte piece per thread.
+template <int KIND>
+__global__ void __launch_bounds__(256) pack_mma_codes_kernel(const uint8_t* __restrict__ q, int E,
+                                                             uint8_t* __restrict__ out) {
+  using D = F4Dims<KIND>;
+  const int64_t pieces = (int64_t)E * D::NJ * D::KCH * kF4Rows * 8;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < pieces; w += (int64_t)gridDim.x * blockDim.x) {
+    const int piece = (int)(w & 7);                  // physical 16-byte piece of the row
+    const int L = (int)((w >> 3) % kF4Rows);
+    const int64_t blk = (w >> 3) / kF4Rows;          // (e, j, c)
+    const int c = (int)(blk % D::KCH);
+    const int64_t ej = blk / D::KCH;
+    const int j = (int)(ej % D::NJ), e = (int)(ej / D::NJ);
+    const int k = c * 128 + ((piece ^ L) & 7) * 16;  // logical K byte of this piece
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (k < D::KB) v = *reinterpret_cast<const uint4*>(q + (size_t)f4_tile_row<KIND>(e, j, L) * D::KB + k);
+    *reinterpret_cast<uint4*>(out + (blk * kF4Rows + L) * 128 + piece * 16) = v;
+  }
+}
+
 // ------------------------------------------------------------ scale packing
 // out[((e NJ + j) KS + q) 512 + 16 r0 + 4 r1 + i] = s[row(e, j, r0 + 32 r1), 4 q + i]:
 // one 32-bit word (the 4 scales of one row and K step) per thread.
@@ -213,52 +251,89 @@ __global__ void __launch_bounds__(256) pack_mma_scales_kernel(const uint8_t* __r
 }
 
 // ---------------------------------------------------- activation quantising
-// x[token of padded row R] -> codes aq[R] and scale chunks asf, one 16-element
-// block per thread under the static global gx; padded rows get zero codes and
-// scales.
+// Padded row of sorted position pos: the tile start of its expert plus its
+// rank within the expert (prefix = token tiles per expert, offsets = slots).
+__device__ __forceinline__ int padded_row(const int* prefix, const int* meta, int nt, int pos) {
+  int lo = 0, hi = kE - 1;  // largest e with offsets[e] <= pos
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (meta[kMetaOffsets + mid] <= pos) lo = mid; else hi = mid - 1;
+  }
+  return prefix[lo] * nt + (pos - meta[kMetaOffsets + lo]);
+}
+
+// Each token's x quantised once under the static global gx (one warp per
+// token, one 16-element block per lane and step), its codes and scales
+// written to the padded rows of its 8 slots, and each slot's routing weight
+// to its padded row.  Padding rows are left as they are: a padding row only
+// feeds its own (unused) accumulator column.
 template <int NT>
 __global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restrict__ x, const int* __restrict__ meta,
-                                                        const int* __restrict__ sorted_slot, int T, int spt, float gx,
-                                                        uint8_t* __restrict__ aq, uint8_t* __restrict__ asf,
+                                                        const int* __restrict__ slot_pos, int T, float gx,
+                                                        const float* __restrict__ wts, uint8_t* __restrict__ aq,
+                                                        uint8_t* __restrict__ asf, float* __restrict__ roww,
                                                         int* status) {
   constexpr int NB = kH / kBlock;  // 176 blocks per row
   constexpr int KS = kH / 64;
+  constexpr int KCH = kH / 256;
   __shared__ int prefix[kE + 1];
   if (threadIdx.x < 32) tile_prefix_warp(meta, NT, prefix);
   __syncthreads();
+  const int lane = threadIdx.x & 31;
   const TensorScale ts = scale_consts(gx);
-  const int64_t total = (int64_t)prefix[kE] * NT * NB;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int R = (int)(idx / NB), kb = (int)(idx % NB);
-    const int tile = R / NT, r = R % NT;
-    const int e = expert_of_tile(prefix, tile);
-    const int n = (tile - prefix[e]) * NT + r;
-    const int off = meta[kMetaOffsets + e], cnt = meta[kMetaOffsets + e + 1] - off;
-    uint2 codes = make_uint2(0u, 0u);
-    uint32_t sc = 0;
-    if (n < cnt) {
-      int tok = sorted_slot[off + n] / spt;
-      if (tok < 0 || tok >= T) {
+  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+    // lanes 0..7: the padded row of slot j = lane (-1: a position outside the permutation)
+    int R = 0;
+    if (lane < kTopK) {
+      const int pos = slot_pos[t * kTopK + lane];
+      if (pos < 0 || pos >= meta[kMetaOffsets + kE]) {
         record_status(status, kStatusDevice);
-        tok = 0;
+        R = -1;
+      } else {
+        R = padded_row(prefix, meta, NT, pos);
+        roww[R] = wts[t * kTopK + lane];
       }
-      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * kH + kb * kBlock);
-      const uint4 v0 = ldg_nc_v4(src), v1 = ldg_nc_v4(src + 1);
-      const uint32_t pr[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      float xv[16];
-      uint32_t key2 = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        xv[2 * k] = bf16_bits_to_f32(pr[k] & 0xFFFFu);
-        xv[2 * k + 1] = bf16_bits_to_f32(pr[k] >> 16);
-        key2 = __vmaxu2(key2, pr[k] & 0x7FFF7FFFu);
-      }
-      const float amax = bf16_bits_to_f32(max(key2 & 0xFFFFu, key2 >> 16));
-      sc = encode_block16f(xv, amax, ts, codes);
     }
-    *reinterpret_cast<uint2*>(aq + (size_t)R * (kH / 2) + kb * 8) = codes;
-    asf[((size_t)tile * KS + (kb >> 2)) * kSfChunk + 16 * (r & 31) + 4 * (r >> 5) + (kb & 3)] = (uint8_t)sc;
+    int rows[kTopK];
+#pragma unroll
+    for (int j = 0; j < kTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, R, j);
+    for (int kb = lane; kb < NB + 16; kb += 32) {
+      // 192 lanes-steps: the last 16 lanes of the last step only gather scales
+      uint2 codes = make_uint2(0u, 0u);
+      uint32_t sc = 0;
+      if (kb < NB) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * kH + kb * kBlock);
+        const uint4 v0 = ldg_nc_v4(src), v1 = ldg_nc_v4(src + 1);
+        const uint32_t pr[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float xv[16];
+        uint32_t key2 = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          xv[2 * k] = bf16_bits_to_f32(pr[k] & 0xFFFFu);
+          xv[2 * k + 1] = bf16_bits_to_f32(pr[k] >> 16);
+          key2 = __vmaxu2(key2, pr[k] & 0x7FFF7FFFu);
+        }
+        sc = encode_block16f(xv, bf16_bits_to_f32(max(key2 & 0xFFFFu, key2 >> 16)), ts, codes);
+      }
+      // the 4 scales of one MMA K step (lanes 4g..4g+3) as one word in lane 4g
+      uint32_t word = sc;
+      word |= __shfl_down_sync(0xffffffffu, sc, 1) << 8;
+      word |= __shfl_down_sync(0xffffffffu, sc, 2) << 16;
+      word |= __shfl_down_sync(0xffffffffu, sc, 3) << 24;
+      if (kb < NB) {
+#pragma unroll
+        for (int j = 0; j < kTopK; ++j) {
+          const int Rj = rows[j];
+          if (Rj < 0) continue;
+          const int tile = Rj / NT, r = Rj % NT;
+          const int c = kb >> 4, kbyte = (kb & 15) * 8;
+          *reinterpret_cast<uint2*>(aq + ((size_t)tile * KCH + c) * (NT * 128) + sw128(r, kbyte)) = codes;
+          if ((kb & 3) == 0)
+            *reinterpret_cast<uint32_t*>(asf + ((size_t)tile * KS + (kb >> 2)) * kSfChunk + 16 * (r & 31) + 4 * (r >> 5)) =
+                word;
+        }
+      }
+    }
   }
 }
 
@@ -272,8 +347,8 @@ __device__ __forceinline__ bool f4_wait(F4Smem<KIND, NT>& sm, uint64_t* bar, uin
 }
 
 template <int KIND, int NT>
-__global__ void __launch_bounds__(kF4Threads, 1)
-    fp4_moe_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, W4A4Args p) {
+__global__ void __launch_bounds__(F4Cfg<KIND, NT>::THREADS, 1)
+    fp4_moe_kernel(W4A4Args p) {
   using C = F4Cfg<KIND, NT>;
   using D = F4Dims<KIND>;
   using Smem = F4Smem<KIND, NT>;
@@ -286,13 +361,15 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     if (lane == 0) {
       for (int s = 0; s < C::NS; ++s) {
         mbar_init(&sm.full[s], 1);
+        mbar_init(&sm.sf_ready[s], 1);
         mbar_init(&sm.empty[s], 1);
       }
       for (int b = 0; b < 2; ++b) {
         mbar_init(&sm.d_full[b], 1);
-        mbar_init(&sm.d_empty[b], 4);  // one arrival per epilogue warp
+        mbar_init(&sm.d_empty[b], 4 * C::NEPI);  // one arrival per epilogue warp
       }
       mbar_init(&sm.fin, 1);
+      mbar_init(&sm.sf_fin, 1);
       sm.abort_flag = 0;
       sm.issued_chunks = 0;
       fence_mbar_init();
@@ -321,15 +398,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           if (use > 0 && !f4_wait(sm, &sm.empty[s], (use - 1) & 1, p.status)) { ok = false; break; }
           const int nks = min(4, D::KS - 4 * c);
           mbar_arrive_expect_tx(&sm.full[s], C::A_BYTES + C::B_BYTES + 2 * nks * kSfChunk);
-          if (KIND == 0) {
-            // 8 boxes of 16 rows: box b = gate (b even) or up rows of units 16 (b / 2)..
-#pragma unroll
-            for (int b = 0; b < 8; ++b)
-              tma_load_2d(smem_u32(sm.a[s]) + b * 2048, &tm_a, c * 128, f4_tile_row<KIND>(e, j, 16 * b), &sm.full[s]);
-          } else {
-            tma_load_2d(smem_u32(sm.a[s]), &tm_a, c * 128, f4_tile_row<KIND>(e, j, 0), &sm.full[s]);
-          }
-          tma_load_2d(smem_u32(sm.b[s]), &tm_b, c * 128, mt * NT, &sm.full[s]);
+          bulk_g2s(sm.a[s], p.wq + ((size_t)(e * D::NJ + j) * D::KCH + c) * C::A_BYTES, C::A_BYTES, &sm.full[s]);
+          bulk_g2s(sm.b[s], p.aq + ((size_t)mt * D::KCH + c) * C::B_BYTES, C::B_BYTES, &sm.full[s]);
           bulk_g2s(sm.sfa[s], p.wsf + ((size_t)(e * D::NJ + j) * D::KS + 4 * c) * kSfChunk, nks * kSfChunk,
                    &sm.full[s]);
           bulk_g2s(sm.sfb[s], p.asf + ((size_t)mt * D::KS + 4 * c) * kSfChunk, nks * kSfChunk, &sm.full[s]);
@@ -337,8 +407,33 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         }
       }
     }
+  } else if (warp == kF4Sf) {
+    // ------------------------------------------- block scales -> tensor memory
+    // per stage: one 32 x 128-bit copy per K step and operand into the
+    // stage's own columns, then a commit that tells the MMA warp they landed
+    uint32_t kiter = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      for (int c = 0; c < D::KCH; ++c, ++kiter) {
+        const int s = kiter % C::NS, use = kiter / C::NS;
+        ok = f4_wait(sm, &sm.full[s], use & 1, p.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        const int nks = min(4, D::KS - 4 * c);
+        const uint32_t sfa_t = taddr + (uint32_t)(C::SF_COL0 + 32 * s), sfb_t = sfa_t + 16;
+        for (int q = 0; q < nks; ++q) {
+          tc_cp_sf_warp(sfa_t + 4 * q, make_sf_desc(smem_u32(sm.sfa[s]) + q * kSfChunk));
+          tc_cp_sf_warp(sfb_t + 4 * q, make_sf_desc(smem_u32(sm.sfb[s]) + q * kSfChunk));
+        }
+        tc_commit_warp_f4(&sm.sf_ready[s]);
+      }
+    }
+    tc_commit_warp_f4(&sm.sf_fin);
+    mbar_wait_bounded(&sm.sf_fin, 0);
+    __syncwarp();
   } else if (warp == kF4Mma) {
-    // ------------------------------------------------- scale copies and MMAs
+    // ----------------------------------------------------------------- MMAs
     uint32_t kiter = 0, titer = 0;
     bool ok = true;
     constexpr uint32_t idesc = make_idesc_mxf4(kF4Rows, NT);
@@ -351,7 +446,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       const uint32_t d = taddr + (uint32_t)(db * NT);
       for (int c = 0; c < D::KCH; ++c, ++kiter) {
         const int s = kiter % C::NS, use = kiter / C::NS;
-        ok = f4_wait(sm, &sm.full[s], use & 1, p.status);
+        ok = f4_wait(sm, &sm.full[s], use & 1, p.status) && f4_wait(sm, &sm.sf_ready[s], use & 1, p.status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
@@ -359,8 +454,6 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         const uint32_t sfa_t = taddr + (uint32_t)(C::SF_COL0 + 32 * s), sfb_t = sfa_t + 16;
         const uint64_t ad = make_sw128_desc(smem_u32(sm.a[s])), bd = make_sw128_desc(smem_u32(sm.b[s]));
         for (int q = 0; q < nks; ++q) {
-          tc_cp_sf_warp(sfa_t + 4 * q, make_sf_desc(smem_u32(sm.sfa[s]) + q * kSfChunk));
-          tc_cp_sf_warp(sfb_t + 4 * q, make_sf_desc(smem_u32(sm.sfb[s]) + q * kSfChunk));
           // K step q: 64 codes = 32 bytes further along the swizzled rows
           tc_mma_fp4_warp(d, ad + (uint64_t)(2 * q), bd + (uint64_t)(2 * q), idesc, sfa_t + 4 * q, sfb_t + 4 * q,
                           c != 0 || q != 0);
@@ -375,32 +468,48 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     __syncwarp();
   } else if (warp >= kF4Epi0) {
     // ------------------------------------------------------------ epilogue
-    const int qd = warp - kF4Epi0;  // lane quarter of tensor memory
+    constexpr int TPS = C::TPS, PW = (TPS + 31) / 32;
+    const int qd = warp & 3;                  // tensor-memory lane quarter
+    const int ew = warp - kF4Epi0;            // epilogue warp 0 .. 4 NEPI - 1
+    const int n0 = (ew >> 2) * TPS;           // this set's first token column
     const TensorScale tsh = scale_consts(p.gh);
+    // the tile's expert, token range, global and (down) per-token weights,
+    // loaded one tile ahead so that their latency hides behind the previous tile
+    struct TileMeta {
+      int mt, j, e, off, cnt;
+      float g;
+      float w[PW];
+    };
+    auto load_meta = [&](int t) {
+      TileMeta m;
+      m.mt = t / D::NJ;
+      m.j = t % D::NJ;
+      m.e = expert_of_tile(sm.mt_prefix, m.mt);
+      m.off = __ldg(p.meta + kMetaOffsets + m.e);
+      m.cnt = __ldg(p.meta + kMetaOffsets + m.e + 1) - m.off;
+      m.g = __ldg(p.wg + m.e) * p.gin;
+#pragma unroll
+      for (int i = 0; i < PW; ++i)
+        m.w[i] = (KIND == 1 && lane + 32 * i < TPS) ? __ldg(p.roww + (size_t)m.mt * NT + n0 + lane + 32 * i) : 0.f;
+      return m;
+    };
+    TileMeta nxt;
+    if ((int)blockIdx.x < n_tiles) nxt = load_meta(blockIdx.x);
     uint32_t titer = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++titer) {
-      const int mt = t / D::NJ, j = t % D::NJ;
-      const int e = expert_of_tile(sm.mt_prefix, mt);
-      const int i = mt - sm.mt_prefix[e];
-      const int off = p.meta[kMetaOffsets + e], cnt = p.meta[kMetaOffsets + e + 1] - off;
-      const int nvalid = min(NT, cnt - i * NT), pos0 = off + i * NT;
+      const TileMeta cur = nxt;
+      if (t + (int)gridDim.x < n_tiles) nxt = load_meta(t + gridDim.x);
+      const int i = cur.mt - sm.mt_prefix[cur.e];
+      const int nvalid = min(NT, cur.cnt - i * NT), pos0 = cur.off + i * NT;
+      const int nend = min(nvalid, n0 + TPS);  // this set's valid columns: n0 .. nend - 1
       const int db = titer & 1, duse = titer >> 1;
-      if (KIND == 1) {
-        // per token column: routing weight x G_d x Gh (before the accumulator wait)
-        __syncwarp();
-        const float G = p.wg[e] * p.gin;
-        for (int n = lane; n < NT; n += 32)
-          sm.tokw[qd][n] = n < nvalid ? __ldg(p.wts + __ldg(p.sorted_slot + pos0 + n)) * G : 0.f;
-        __syncwarp();
-      }
       if (!f4_wait(sm, &sm.d_full[db], duse & 1, p.status)) break;
       tc_fence_after();
       const uint32_t trow = taddr + ((uint32_t)(qd * 32) << 16) + (uint32_t)(db * NT);
       if (KIND == 0) {
-        float* stg = sm.stage[qd];
-        const float G = p.gin * p.wg[e];
+        float* stg = sm.stage[ew];
         const bool up = lane >= 16;
-        for (int cc = 0; cc * 16 < nvalid; ++cc) {
+        for (int cc = n0 / 16; cc * 16 < nend; ++cc) {
           float v[16], o[16];
           tmem_ld16(trow + cc * 16, v);
 #pragma unroll
@@ -411,19 +520,19 @@ __global__ void __launch_bounds__(kF4Threads, 1)
             const float g = up ? o[k + 8] : v[k];
             const float u = up ? v[k + 8] : o[k];
             const int n = cc * 16 + (up ? k + 8 : k);
-            stg[n * 16 + (lane & 15)] = gelu_tanh(G * g) * (G * u);
+            stg[(n - n0) * 16 + (lane & 15)] = gelu_tanh(cur.g * g) * (cur.g * u);
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.d_empty[db]);
         // quantise: one token's 16 hidden units per lane
-        for (int n = lane; n < NT; n += 32) {
+        for (int n = n0 + lane; n < n0 + TPS; n += 32) {
           uint2 codes = make_uint2(0u, 0u);
           uint32_t sc = 0;
           if (n < nvalid) {
             float hv[16];
-            const float4* src = reinterpret_cast<const float4*>(stg + n * 16);
+            const float4* src = reinterpret_cast<const float4*>(stg + (n - n0) * 16);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const float4 f = src[k];
@@ -434,22 +543,28 @@ __global__ void __launch_bounds__(kF4Threads, 1)
             for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(hv[k]));
             sc = encode_block16f(hv, amax, tsh, codes);
           }
-          const size_t R = (size_t)mt * NT + n;
-          *reinterpret_cast<uint2*>(p.hq + R * (kI / 2) + j * 32 + qd * 8) = codes;
-          p.hsf[((size_t)mt * (kI / 64) + j) * kSfChunk + 16 * (n & 31) + 4 * (n >> 5) + qd] = (uint8_t)sc;
+          // K byte 32 j + 8 qd of the hidden row: chunk (32 j + 8 qd) / 128 of the down operand
+          const int kbyte = cur.j * 32 + qd * 8;
+          *reinterpret_cast<uint2*>(p.hq + ((size_t)cur.mt * F4Dims<1>::KCH + (kbyte >> 7)) * (NT * 128) +
+                                    sw128(n, kbyte & 127)) = codes;
+          p.hsf[((size_t)cur.mt * (kI / 64) + cur.j) * kSfChunk + 16 * (n & 31) + 4 * (n >> 5) + qd] = (uint8_t)sc;
         }
         __syncwarp();
       } else {
         // lane = output row; per token one 4-byte store per lane (128 bytes per warp)
-        const int row = j * kF4Rows + qd * 32 + lane;
+        const int row = cur.j * kF4Rows + qd * 32 + lane;
         constexpr int CW = NT % 32 == 0 ? 32 : 16;
-        for (int cc = 0; cc * CW < nvalid; ++cc) {
+        for (int cc = n0 / CW; cc * CW < nend; ++cc) {
           float v[CW];
           if constexpr (CW == 32) tmem_ld32(trow + cc * CW, v); else tmem_ld16(trow + cc * CW, v);
           const int nmax = min(CW, nvalid - cc * CW);
+          const int ln = cc * CW - n0;          // first column of the chunk within the set
+          const float wr = (ln >> 5) == 0 ? cur.w[0] : cur.w[PW - 1];
 #pragma unroll
-          for (int k = 0; k < CW; ++k)
-            if (k < nmax) p.obuf[(size_t)(pos0 + cc * CW + k) * kH + row] = v[k] * sm.tokw[qd][cc * CW + k];
+          for (int k = 0; k < CW; ++k) {
+            const float wk = __shfl_sync(0xffffffffu, wr, (ln & 31) + k) * cur.g;
+            if (k < nmax) p.obuf[(size_t)(pos0 + cc * CW + k) * kH + row] = v[k] * wk;
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -474,27 +589,22 @@ __global__ void __launch_bounds__(kF4Threads, 1)
 
 template <int KIND, int NT>
 cudaError_t launch_fp4(const W4A4Args& a, cudaStream_t st) {
-  using D = F4Dims<KIND>;
   static_assert(sizeof(F4Smem<KIND, NT>) + 1024 <= 232448, "shared memory budget");
   const int smem = (int)sizeof(F4Smem<KIND, NT>) + 1024;
   cudaError_t err = configure_kernel_once((const void*)fp4_moe_kernel<KIND, NT>, smem);
   if (err != cudaSuccess) return err;
-  CUtensorMap tm_a, tm_b;
-  const uint64_t wrows = (uint64_t)kE * (KIND == 0 ? 2 * kI : kH);
-  const bool ok =
-      encode_tma_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.wq, D::KB, wrows, D::KB, 128, KIND == 0 ? 16 : 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B) &&
-      encode_tma_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.aq, D::KB, (uint64_t)a.max_tiles * NT, D::KB, 128, NT,
-                    CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return cudaErrorInvalidValue;
   int sms = 0;
   err = sm_count(&sms);
   if (err != cudaSuccess) return err;
-  fp4_moe_kernel<KIND, NT><<<sms, kF4Threads, smem, st>>>(tm_a, tm_b, a);
+  fp4_moe_kernel<KIND, NT><<<sms, F4Cfg<KIND, NT>::THREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+size_t w4a4_packed_code_bytes(int E, int kind) {
+  return (size_t)E * (kind == 0 ? F4Dims<0>::NJ * F4Dims<0>::KCH : F4Dims<1>::NJ * F4Dims<1>::KCH) * kF4Rows * 128;
+}
 
 int w4a4_tile_tokens(int T) { return T <= 256 ? 16 : (T <= 1024 ? 64 : 128); }
 
@@ -507,14 +617,23 @@ cudaError_t launch_w4a4_pack_scales(const uint8_t* s, int E, int kind, uint8_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_w4a4_act_quant(const uint16_t* x, const int* meta, const int* sorted_slot, int T, int spt, float gx,
-                                  int nt, int max_tiles, uint8_t* aq, uint8_t* asf, int* status, cudaStream_t st) {
-  const int64_t work = (int64_t)max_tiles * nt * (kH / kBlock);
-  const int blocks = (int)std::min<int64_t>((work + 255) / 256, 148 * 16);
+cudaError_t launch_w4a4_pack_codes(const uint8_t* q, int E, int kind, uint8_t* out, cudaStream_t st) {
+  const int64_t pieces = (int64_t)E * (kind == 0 ? F4Dims<0>::NJ * F4Dims<0>::KCH : F4Dims<1>::NJ * F4Dims<1>::KCH) *
+                         kF4Rows * 8;
+  const int blocks = (int)std::min<int64_t>((pieces + 255) / 256, 148 * 16);
+  if (kind == 0) pack_mma_codes_kernel<0><<<blocks, 256, 0, st>>>(q, E, out);
+  else pack_mma_codes_kernel<1><<<blocks, 256, 0, st>>>(q, E, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_w4a4_act_quant(const uint16_t* x, const int* meta, const int* slot_pos, const float* wts, int T,
+                                  float gx, int nt, uint8_t* aq, uint8_t* asf, float* roww, int* status,
+                                  cudaStream_t st) {
+  const int blocks = (int)std::min<int64_t>((T + 7) / 8, 148 * 8);
   switch (nt) {
-    case 16: act_quant_kernel<16><<<blocks, 256, 0, st>>>(x, meta, sorted_slot, T, spt, gx, aq, asf, status); break;
-    case 64: act_quant_kernel<64><<<blocks, 256, 0, st>>>(x, meta, sorted_slot, T, spt, gx, aq, asf, status); break;
-    case 128: act_quant_kernel<128><<<blocks, 256, 0, st>>>(x, meta, sorted_slot, T, spt, gx, aq, asf, status); break;
+    case 16: act_quant_kernel<16><<<blocks, 256, 0, st>>>(x, meta, slot_pos, T, gx, wts, aq, asf, roww, status); break;
+    case 64: act_quant_kernel<64><<<blocks, 256, 0, st>>>(x, meta, slot_pos, T, gx, wts, aq, asf, roww, status); break;
+    case 128: act_quant_kernel<128><<<blocks, 256, 0, st>>>(x, meta, slot_pos, T, gx, wts, aq, asf, roww, status); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

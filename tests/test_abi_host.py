@@ -220,15 +220,17 @@ def test_aff4_validation(capi):
 
 
 def _w4a4(c, gx=0.003, gh=0.0007, sf=4096):
-    return c.moe_experts_w4a4(_experts(c), sf, sf, gx, gh)
+    return c.moe_experts_w4a4(_experts(c), sf, sf, sf, sf, gx, gh)
 
 
 def test_w4a4_validation(capi):
     c = capi
     r, w = _router(c), _w4a4(c)
-    assert c.moe_w4a4_scale_bytes(128, 0) == 128 * 1408 * 176
-    assert c.moe_w4a4_scale_bytes(128, 1) == 128 * 2816 * 44
-    assert c.moe_w4a4_scale_bytes(0, 0) == 0 and c.moe_w4a4_scale_bytes(128, 2) == 0
+    assert c.moe_w4a4_pack_bytes(128, 0) == 128 * 11 * 11 * 128 * 128      # 128-row tiles x 256-element chunks
+    assert c.moe_w4a4_pack_bytes(128, 1) == 128 * 22 * 3 * 128 * 128
+    assert c.moe_w4a4_pack_bytes(128, 2) == 128 * 1408 * 176
+    assert c.moe_w4a4_pack_bytes(128, 3) == 128 * 2816 * 44
+    assert c.moe_w4a4_pack_bytes(0, 0) == 0 and c.moe_w4a4_pack_bytes(128, 4) == 0
     sizes = [c.moe_w4a4_workspace_bytes(T, ctypes.byref(w), ctypes.byref(r)) for T in (1, 64, 4096)]
     assert 0 < sizes[0] < sizes[1] < sizes[2]
     assert c.moe_w4a4_workspace_bytes(65537, ctypes.byref(w), ctypes.byref(r)) == 0
@@ -245,5 +247,6 @@ def test_w4a4_validation(capi):
     assert c.moe_w4a4_forward(P, 1, ctypes.byref(_w4a4(c, sf=4096 + 8)), ctypes.byref(r), P, P, n,
                               None) == c.NVFP4_ERR_ALIGNMENT
     x = _experts(c, I=512)
-    assert c.moe_w4a4_pack_scales(ctypes.byref(x), P, P, None) == c.NVFP4_ERR_UNSUPPORTED
-    assert c.moe_w4a4_pack_scales(ctypes.byref(_experts(c)), None, P, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_w4a4_pack(ctypes.byref(x), P, P, P, P, None) == c.NVFP4_ERR_UNSUPPORTED
+    assert c.moe_w4a4_pack(ctypes.byref(_experts(c)), None, P, P, P, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_w4a4_pack(ctypes.byref(_experts(c)), P, P, P + 4, P, None) == c.NVFP4_ERR_ALIGNMENT

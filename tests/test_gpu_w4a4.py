@@ -3,7 +3,7 @@ on the GPU against the W4A4 oracle.
 
 What is unique is compared exactly; where a floating-point sum decides an
 integer the comparison allows what that sum may legitimately decide:
-  * packed weight scales: bit-exact against the documented chunk layout;
+  * packed weight codes and scales: bit-exact against the documented layouts;
   * x codes and scales: bit-exact (both sides quantise the same bf16 values
     with the same fp32 steps);
   * hidden codes and scales: the GPU forms h from fp32 tensor-core sums, the
@@ -47,6 +47,18 @@ def _padded_rows(counts, offsets, nt):
     return rows
 
 
+def _swizzled_rows(buf, rows, nt, nchunk, nbytes):
+    """Rows [len(rows), nbytes] of codes stored tile-major in 128-byte swizzled
+    blocks (tile p, chunk c: nt rows of 128 bytes; byte k of row r at
+    128 r + 16 ((k / 16) ^ (r % 8)) + k % 16)."""
+    k = np.arange(nchunk * 128)
+    c, kk = k // 128, k % 128
+    tile, r = rows // nt, rows % nt
+    idx = ((tile[:, None] * nchunk + c[None, :]) * nt + r[:, None]) * 128 \
+        + 16 * ((kk[None, :] // 16) ^ (r[:, None] % 8)) + kk[None, :] % 16
+    return buf[idx][:, :nbytes]
+
+
 def _chunk_scales(chunks, rows, nt, K):
     """Scales [len(rows), K/16] of the given padded rows from the 512-byte chunks."""
     g = K // 64
@@ -56,22 +68,30 @@ def _chunk_scales(chunks, rows, nt, K):
     return chunks[idx]
 
 
-def test_pack_scales_layout(layer, layer0):
-    """Chunk (e, j, q): byte 16 r0 + 4 r1 + i = scale of tile row r0 + 32 r1,
-    block 4 q + i; gate_up tile rows interleave the gate and up rows of 16
-    hidden units per lane quarter."""
+def test_pack_layout(layer, layer0):
+    """Codes: block (e, j, c) holds tile rows L of K bytes 128 c.. in the
+    128-byte swizzle; scales: chunk (e, j, q) byte 16 r0 + 4 r1 + i = scale of
+    tile row r0 + 32 r1, block 4 q + i; gate_up tile rows interleave the gate
+    and up rows of 16 hidden units per lane quarter."""
     ex = layer0["ex"]
+    Lq = np.arange(128)
+    qd, w = Lq >> 5, Lq & 31
+    gu_pk = layer.gate_up_pk.cpu().numpy().reshape(E, 11, 11 * 128 * 128)
+    dn_pk = layer.down_pk.cpu().numpy().reshape(E, 22, 3 * 128 * 128)
     gu = layer.gate_up_sf.cpu().numpy().reshape(E, 11, 44, 32, 4, 4)   # e, j, q, r0, r1, i
     dn = layer.down_sf.cpu().numpy().reshape(E, 22, 11, 32, 4, 4)
     L = np.arange(128).reshape(4, 32).T           # [r0, r1] -> tile row
-    qd, w = L >> 5, L & 31
     for e in (0, 77, 127):
         for j in (0, 5, 10):
             grow = np.where(w < 16, 0, I) + j * 64 + qd * 16 + (w & 15)
-            want = ex.gate_up_s[e][grow]                      # [32, 4, 176]
-            want = want.reshape(32, 4, 44, 4).transpose(2, 0, 1, 3)
+            assert np.array_equal(_swizzled_rows(gu_pk[e, j], Lq, 128, 11, H // 2), ex.gate_up_q[e][grow])
+            grow2 = grow[L]
+            want = ex.gate_up_s[e][grow2].reshape(32, 4, 44, 4).transpose(2, 0, 1, 3)
             assert np.array_equal(gu[e, j], want)
         for j in (0, 13, 21):
+            got = _swizzled_rows(dn_pk[e, j], Lq, 128, 3, 384)
+            assert np.array_equal(got[:, :I // 2], ex.down_q[e][j * 128 + Lq])
+            assert not got[:, I // 2:].any()
             want = ex.down_s[e][j * 128 + L].reshape(32, 4, 11, 4).transpose(2, 0, 1, 3)
             assert np.array_equal(dn[e, j], want)
 
@@ -126,11 +146,11 @@ def test_w4a4_forward(layer, layer0, dev, T):
     prow = rows_of_pos[v["slot_pos"][slots]]
     xq = np.repeat(ref["xq"], K8, axis=0)
     xs = np.repeat(ref["xs"], K8, axis=0)
-    assert np.array_equal(v["x_codes"][prow], xq)
+    assert np.array_equal(_swizzled_rows(v["x_codes"], prow, nt, 11, H // 2), xq)
     assert np.array_equal(_chunk_scales(v["x_scales"], prow, nt, H), xs)
 
     # hidden codes: rare, valid threshold decisions only
-    hq_gpu = v["h_codes"][prow]
+    hq_gpu = _swizzled_rows(v["h_codes"], prow, nt, 3, I // 2)
     hs_gpu = _chunk_scales(v["h_scales"], prow, nt, I)
     local = (np.arange(len(toks))[:, None] * K8 + np.arange(K8)[None, :]).ravel()
     hq_ref, hs_ref, h32 = ref["hq"][local], ref["hs"][local], ref["h32"][local]
@@ -149,7 +169,7 @@ def test_w4a4_forward(layer, layer0, dev, T):
     assert rel <= 4e-3 and mx <= 4e-2, (rel, mx)
 
 
-def test_w4a4_padding_rows_are_zero(layer, dev):
+def test_w4a4_hidden_padding_rows_are_zero(layer, dev):
     T = 24
     x = gen.make_x(950, T)
     _, v = _run(layer, dev, x)
@@ -159,8 +179,7 @@ def test_w4a4_padding_rows_are_zero(layer, dev):
     total = int(((counts + nt - 1) // nt).sum()) * nt
     pad = np.setdiff1d(np.arange(total), rows)
     assert pad.size > 0
-    assert not v["x_codes"][pad].any() and not v["h_codes"][pad].any()
-    assert not _chunk_scales(v["x_scales"], pad, nt, H).any()
+    assert not _swizzled_rows(v["h_codes"], pad, nt, 3, I // 2).any()
     assert not _chunk_scales(v["h_scales"], pad, nt, I).any()
 
 
