@@ -285,12 +285,14 @@ class _Ctx:
         self._experts = {}
 
     def experts(self, seed):
-        """Device copy of a layer's experts (shared by workloads on the same seed)."""
+        """Device copy of a layer's experts with their packed code tiles (made
+        once at load, like the quantisation itself; the decode kernels stream
+        them as whole blocks), shared by workloads on the same seed."""
         import moe_inputs as gen
         import nvfp4_weight_only_router_b200 as lib
         if seed not in self._experts:
             ex = gen.make_experts(seed)
-            self._experts[seed] = lib.Experts.from_host(ex, self.dev)
+            self._experts[seed] = lib.Experts.from_host(ex, self.dev).packed()
             del ex
         return self._experts[seed]
 
@@ -634,7 +636,8 @@ def measure(ctx, workload, args, cpu_baseline=True):
         "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
         "config": {"workload": workload, "desc": wl["desc"], "T": T,
                    "l2": "256 MiB flush write between timed steps",
-                   "graph": workload != "quantize", "parallelism": f"replicas x{world}"},
+                   "graph": workload != "quantize", "parallelism": f"replicas x{world}",
+                   "weights": None if workload == "quantize" or wl.get("aff4") else "NVFP4 codes + packed 16 KB code tiles"},
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": kernels_per_step * args.steps, "clocks": clocks,
     }

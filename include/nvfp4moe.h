@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define NVFP4MOE_ABI_VERSION 2
+#define NVFP4MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define NVFP4MOE_API __attribute__((visibility("default")))
@@ -86,7 +86,11 @@ typedef struct {
   float eps;                     /* RMSNorm epsilon (the pages are silent; 1e-6) */
 } moe_router;
 
-/* NVFP4 expert stacks.  All pointers are device pointers. */
+/* NVFP4 expert stacks.  All pointers are device pointers.  gate_up_pk and
+ * down_pk are optional (NULL = absent): the same codes copied once by
+ * moe_nvfp4_pack_codes into whole 16 KB tiles, which the decode kernels then
+ * stream as contiguous blocks instead of gathering 128-byte row pieces;
+ * moe_w4a4_forward requires them. */
 typedef struct {
   const uint8_t* gate_up_q;  /* [E, 2I, H/2] */
   const uint8_t* gate_up_s;  /* [E, 2I, H/16] */
@@ -97,7 +101,28 @@ typedef struct {
   int32_t E;                 /* must be 128 */
   int32_t H;                 /* must be 2816 */
   int32_t I;                 /* must be 704 */
+  const uint8_t* gate_up_pk; /* moe_pack_bytes(E, 0) bytes, or NULL */
+  const uint8_t* down_pk;    /* moe_pack_bytes(E, 1) bytes, or NULL */
 } moe_experts;
+
+/* Bytes of the packed gate_up codes (which = 0), down codes (1), gate_up
+ * block scales in the FP4 tensor core's order (2) or down block scales (3)
+ * of E experts (0 for E < 1 or another `which`). */
+NVFP4MOE_API size_t moe_pack_bytes(int32_t E, int32_t which);
+
+/* moe_nvfp4_pack_codes: copies experts->gate_up_q / down_q into
+ * gate_up_pk_dev / down_pk_dev (moe_pack_bytes(E, 0 / 1) bytes, device,
+ * 16-byte aligned, caller-owned): per expert, per 128-row tile of the
+ * projection and per 256 elements of K, the tile's codes as 128 rows of 128
+ * bytes in the 128-byte swizzle (16-byte piece p of tile row r stored at
+ * piece p ^ (r % 8)); bytes past a row's end are zero.  Gate_up tile j holds,
+ * for each quarter q = 0..3, the gate rows of hidden units 64 j + 16 q ..
+ * + 15 followed by their 16 up rows; down tile j holds rows 128 j .. + 127.
+ * Run once per set of weights; asynchronous on `stream`.  Same shape
+ * requirements as moe_nvfp4_forward (the packed pointers of `experts` are
+ * ignored). */
+NVFP4MOE_API nvfp4_status moe_nvfp4_pack_codes(const moe_experts* experts, uint8_t* gate_up_pk_dev,
+                                               uint8_t* down_pk_dev, void* stream);
 
 /* ---------------------------------------------------------------------------
  * nvfp4_quantize: bf16 weights -> NVFP4.
@@ -340,36 +365,27 @@ NVFP4MOE_API nvfp4_status moe_block_forward(const void* x_dev, int32_t T, const 
  * multiplies those codes with the down weights', o = w G_d Gh acc per slot,
  * and y[t] = bf16(sum over the token's 8 slots in slot order).
  *
- * The weights are those of moe_experts, copied once into the tensor core's
- * order by moe_w4a4_pack, so that every pipeline stage reads one contiguous
- * block: per expert, per 128-row tile of the projection (gate_up tiles hold
- * the gate rows of 16 hidden units then their 16 up rows, four times) and
- * per 256 elements of K, the tile's codes as 128 rows of 128 bytes in the
- * 128-byte swizzle (16-byte piece p of row r stored at piece p ^ (r % 8));
- * and per 64 elements of K, the tile's block scales as one 512-byte chunk
- * (row r = r0 + 32 r1 at byte 16 r0 + 4 r1).
+ * The weights are those of moe_experts with their packed codes
+ * (moe_nvfp4_pack_codes), plus their block scales copied once into the FP4
+ * tensor core's order (moe_w4a4_pack_scales): per expert, per 128-row tile
+ * (the packed codes' row order) and per 64 elements of K, one 512-byte chunk,
+ * the scale of tile row r = r0 + 32 r1 and block i of the 64 at byte
+ * 16 r0 + 4 r1 + i.
  * ------------------------------------------------------------------------- */
 typedef struct {
-  moe_experts experts;           /* codes, block scales and globals (moe_nvfp4_forward's) */
-  const uint8_t* gate_up_pk;     /* moe_w4a4_pack_bytes(E, 0) bytes from moe_w4a4_pack */
-  const uint8_t* down_pk;        /* moe_w4a4_pack_bytes(E, 1) bytes */
-  const uint8_t* gate_up_sf;     /* moe_w4a4_pack_bytes(E, 2) bytes */
-  const uint8_t* down_sf;        /* moe_w4a4_pack_bytes(E, 3) bytes */
+  moe_experts experts;           /* moe_nvfp4_forward's, with gate_up_pk and down_pk set */
+  const uint8_t* gate_up_sf;     /* moe_pack_bytes(E, 2) bytes from moe_w4a4_pack_scales */
+  const uint8_t* down_sf;        /* moe_pack_bytes(E, 3) bytes */
   float input_scale_gate_up;     /* Gx > 0, finite */
   float input_scale_down;        /* Gh > 0, finite */
 } moe_experts_w4a4;
 
-/* Bytes of the packed gate_up codes (which = 0), down codes (1), gate_up
- * block scales (2) or down block scales (3) of E experts (0 for E < 1 or
- * another `which`). */
-NVFP4MOE_API size_t moe_w4a4_pack_bytes(int32_t E, int32_t which);
-
-/* moe_w4a4_pack: writes the four packed copies of `experts` (device buffers of
- * moe_w4a4_pack_bytes(E, 0..3) bytes, 16-byte aligned, caller-owned).  Run
- * once per set of weights; asynchronous on `stream`.  Same shape requirements
- * as moe_nvfp4_forward. */
-NVFP4MOE_API nvfp4_status moe_w4a4_pack(const moe_experts* experts, uint8_t* gate_up_pk_dev, uint8_t* down_pk_dev,
-                                        uint8_t* gate_up_sf_dev, uint8_t* down_sf_dev, void* stream);
+/* moe_w4a4_pack_scales: copies experts->gate_up_s / down_s into
+ * gate_up_sf_dev / down_sf_dev (moe_pack_bytes(E, 2 / 3) bytes, device,
+ * 16-byte aligned, caller-owned) in the order above.  Run once per set of
+ * weights; asynchronous on `stream`. */
+NVFP4MOE_API nvfp4_status moe_w4a4_pack_scales(const moe_experts* experts, uint8_t* gate_up_sf_dev,
+                                               uint8_t* down_sf_dev, void* stream);
 
 /* moe_w4a4_forward: y_dev bf16 [T, H] from x_dev bf16 [T, H] as described
  * above; 1 <= T <= 65536, router and experts as for moe_nvfp4_forward.

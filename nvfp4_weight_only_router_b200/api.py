@@ -62,19 +62,37 @@ class Router:
 
 @dataclasses.dataclass
 class Experts:
-    """NVFP4 expert stacks on the device (layouts of include/nvfp4moe.h)."""
+    """NVFP4 expert stacks on the device (layouts of include/nvfp4moe.h), with
+    the optional packed copy of the codes (see packed())."""
     gate_up_q: torch.Tensor
     gate_up_s: torch.Tensor
     gate_up_g: torch.Tensor
     down_q: torch.Tensor
     down_s: torch.Tensor
     down_g: torch.Tensor
+    gate_up_pk: torch.Tensor | None = None
+    down_pk: torch.Tensor | None = None
 
     def c_struct(self) -> capi.moe_experts:
         return capi.moe_experts(_ptr(self.gate_up_q), _ptr(self.gate_up_s), _ptr(self.gate_up_g),
                                 _ptr(self.down_q), _ptr(self.down_s), _ptr(self.down_g),
                                 self.gate_up_q.shape[0], self.gate_up_q.shape[2] * 2,
-                                self.down_q.shape[2] * 2)
+                                self.down_q.shape[2] * 2, _ptr(self.gate_up_pk), _ptr(self.down_pk))
+
+    def packed(self, stream=None) -> "Experts":
+        """The same experts with the packed code tiles (moe_nvfp4_pack_codes)
+        that the decode kernels stream as whole blocks; shares the other
+        tensors."""
+        if self.gate_up_pk is not None:
+            return self
+        E_ = self.gate_up_q.shape[0]
+        dev = self.gate_up_q.device
+        gu = torch.empty(capi.moe_pack_bytes(E_, 0), dtype=torch.uint8, device=dev)
+        dn = torch.empty(capi.moe_pack_bytes(E_, 1), dtype=torch.uint8, device=dev)
+        plain = dataclasses.replace(self, gate_up_pk=None, down_pk=None)
+        check(capi.moe_nvfp4_pack_codes(ctypes.byref(plain.c_struct()), _ptr(gu), _ptr(dn), _stream(stream)),
+              "moe_nvfp4_pack_codes")
+        return dataclasses.replace(self, gate_up_pk=gu, down_pk=dn)
 
     @staticmethod
     def from_host(x, device="cuda") -> "Experts":
@@ -272,16 +290,16 @@ class W4A4Layer:
     for up to `max_tokens` tokens."""
 
     def __init__(self, experts: Experts, router: Router, gx: float, gh: float, max_tokens: int, stream=None):
+        experts = experts.packed(stream)
         self.experts, self.router = experts, router
         dev = experts.gate_up_q.device
         ex = experts.c_struct()
         E_ = experts.gate_up_q.shape[0]
-        self.gate_up_pk, self.down_pk, self.gate_up_sf, self.down_sf = (
-            torch.empty(capi.moe_w4a4_pack_bytes(E_, w), dtype=torch.uint8, device=dev) for w in range(4))
-        check(capi.moe_w4a4_pack(ctypes.byref(ex), _ptr(self.gate_up_pk), _ptr(self.down_pk), _ptr(self.gate_up_sf),
-                                 _ptr(self.down_sf), _stream(stream)), "moe_w4a4_pack")
-        self._xs = capi.moe_experts_w4a4(ex, _ptr(self.gate_up_pk), _ptr(self.down_pk), _ptr(self.gate_up_sf),
-                                         _ptr(self.down_sf), float(gx), float(gh))
+        self.gate_up_sf, self.down_sf = (torch.empty(capi.moe_pack_bytes(E_, w), dtype=torch.uint8, device=dev)
+                                         for w in (2, 3))
+        check(capi.moe_w4a4_pack_scales(ctypes.byref(ex), _ptr(self.gate_up_sf), _ptr(self.down_sf), _stream(stream)),
+              "moe_w4a4_pack_scales")
+        self._xs = capi.moe_experts_w4a4(ex, _ptr(self.gate_up_sf), _ptr(self.down_sf), float(gx), float(gh))
         self._rs = router.c_struct()
         self.max_tokens = int(max_tokens)
         nbytes = capi.moe_w4a4_workspace_bytes(self.max_tokens, ctypes.byref(self._xs), ctypes.byref(self._rs))

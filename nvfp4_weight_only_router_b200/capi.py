@@ -44,7 +44,8 @@ class moe_router(ctypes.Structure):
 class moe_experts(ctypes.Structure):
     _fields_ = [("gate_up_q", c_void_p), ("gate_up_s", c_void_p), ("gate_up_g", c_void_p),
                 ("down_q", c_void_p), ("down_s", c_void_p), ("down_g", c_void_p),
-                ("E", c_int32), ("H", c_int32), ("I", c_int32)]
+                ("E", c_int32), ("H", c_int32), ("I", c_int32),
+                ("gate_up_pk", c_void_p), ("down_pk", c_void_p)]
 
 
 class moe_forward_views(ctypes.Structure):
@@ -67,8 +68,7 @@ class moe_block(ctypes.Structure):
 
 
 class moe_experts_w4a4(ctypes.Structure):
-    _fields_ = [("experts", moe_experts), ("gate_up_pk", c_void_p), ("down_pk", c_void_p),
-                ("gate_up_sf", c_void_p), ("down_sf", c_void_p),
+    _fields_ = [("experts", moe_experts), ("gate_up_sf", c_void_p), ("down_sf", c_void_p),
                 ("input_scale_gate_up", c_float), ("input_scale_down", c_float)]
 
 
@@ -107,8 +107,9 @@ SIGNATURES = {
     "moe_forward_workspace_views": (c_int32, [c_int32, _X, _R, ctypes.POINTER(moe_forward_views)]),
     "moe_block_workspace_bytes": (c_size_t, [c_int32, _B]),
     "moe_block_forward": (c_int32, [c_void_p, c_int32, _B, c_void_p, c_void_p, c_size_t, c_void_p]),
-    "moe_w4a4_pack_bytes": (c_size_t, [c_int32, c_int32]),
-    "moe_w4a4_pack": (c_int32, [_X, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "moe_pack_bytes": (c_size_t, [c_int32, c_int32]),
+    "moe_nvfp4_pack_codes": (c_int32, [_X, c_void_p, c_void_p, c_void_p]),
+    "moe_w4a4_pack_scales": (c_int32, [_X, c_void_p, c_void_p, c_void_p]),
     "moe_w4a4_workspace_bytes": (c_size_t, [c_int32, _W, _R]),
     "moe_w4a4_forward": (c_int32, [c_void_p, c_int32, _W, _R, c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_w4a4_forward_profiled": (c_int32, [c_void_p, c_int32, _W, _R, c_void_p, c_void_p, c_size_t, c_void_p,

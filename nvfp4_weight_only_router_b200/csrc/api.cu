@@ -151,6 +151,9 @@ nvfp4_status check_experts(const moe_experts* x) {
   const void* ps[] = {x->gate_up_q, x->gate_up_s, x->gate_up_g, x->down_q, x->down_s, x->down_g};
   for (const void* p : ps)
     if (!aligned(p, 16)) return NVFP4_ERR_ALIGNMENT;
+  // the packed copies are optional, but both or neither
+  if ((x->gate_up_pk == nullptr) != (x->down_pk == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(x->gate_up_pk, 16) || !aligned(x->down_pk, 16)) return NVFP4_ERR_ALIGNMENT;
   return NVFP4_OK;
 }
 
@@ -158,6 +161,7 @@ nvfp4_status check_experts(const moe_experts* x) {
 struct ExpertPtrs {
   int codec = kCodecNvfp4;
   const uint8_t *gu_q = nullptr, *gu_s = nullptr, *dn_q = nullptr, *dn_s = nullptr;
+  const uint8_t *gu_pk = nullptr, *dn_pk = nullptr;
   const float *gu_g = nullptr, *dn_g = nullptr;
   const uint16_t *gu_b = nullptr, *dn_b = nullptr;
 };
@@ -171,6 +175,8 @@ ExpertPtrs nvfp4_ptrs(const moe_experts* x) {
   e.dn_q = x->down_q;
   e.dn_s = x->down_s;
   e.dn_g = x->down_g;
+  e.gu_pk = x->gate_up_pk;
+  e.dn_pk = x->down_pk;
   return e;
 }
 
@@ -426,6 +432,8 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const ExpertPtrs& ex,
   xa.dn_s = ex.dn_s;
   xa.dn_g = ex.dn_g;
   xa.dn_b = ex.dn_b;
+  xa.gu_pk = ex.gu_pk;
+  xa.dn_pk = ex.dn_pk;
   xa.x = static_cast<const uint16_t*>(x);
   xa.meta = pa.meta;
   xa.sorted_slot = pa.sorted_slot;
@@ -616,40 +624,45 @@ nvfp4_status check_experts_w4a4(const moe_experts_w4a4* x) {
   if (!x) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_experts(&x->experts);
   if (st != NVFP4_OK) return st;
-  if (!x->gate_up_pk || !x->down_pk || !x->gate_up_sf || !x->down_sf) return NVFP4_ERR_INVALID_ARG;
+  if (!x->experts.gate_up_pk || !x->gate_up_sf || !x->down_sf) return NVFP4_ERR_INVALID_ARG;
   const float gs[2] = {x->input_scale_gate_up, x->input_scale_down};
   for (float g : gs)
     if (!(g > 0.f) || !std::isfinite(g)) return NVFP4_ERR_INVALID_ARG;
-  const void* ps[] = {x->gate_up_pk, x->down_pk, x->gate_up_sf, x->down_sf};
-  for (const void* p : ps)
-    if (!aligned(p, 16)) return NVFP4_ERR_ALIGNMENT;
+  if (!aligned(x->gate_up_sf, 16) || !aligned(x->down_sf, 16)) return NVFP4_ERR_ALIGNMENT;
   return NVFP4_OK;
 }
 
 }  // namespace
 
-size_t moe_w4a4_pack_bytes(int32_t E, int32_t which) {
+size_t moe_pack_bytes(int32_t E, int32_t which) {
   if (E < 1 || E > (1 << 20)) return 0;
   switch (which) {
-    case 0: return w4a4_packed_code_bytes(E, 0);
-    case 1: return w4a4_packed_code_bytes(E, 1);
+    case 0: return packed_code_bytes(E, 0);
+    case 1: return packed_code_bytes(E, 1);
     case 2: return (size_t)E * (2 * kI) * (kH / kBlock);
     case 3: return (size_t)E * kH * (kI / kBlock);
   }
   return 0;
 }
 
-nvfp4_status moe_w4a4_pack(const moe_experts* ex, uint8_t* gu_pk, uint8_t* dn_pk, uint8_t* gu_sf, uint8_t* dn_sf,
-                           void* stream) {
+nvfp4_status moe_nvfp4_pack_codes(const moe_experts* ex, uint8_t* gu_pk, uint8_t* dn_pk, void* stream) {
   nvfp4_status st = check_experts(ex);
   if (st != NVFP4_OK) return st;
-  if (!gu_pk || !dn_pk || !gu_sf || !dn_sf) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned(gu_pk, 16) || !aligned(dn_pk, 16) || !aligned(gu_sf, 16) || !aligned(dn_sf, 16))
-    return NVFP4_ERR_ALIGNMENT;
+  if (!gu_pk || !dn_pk) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(gu_pk, 16) || !aligned(dn_pk, 16)) return NVFP4_ERR_ALIGNMENT;
   cudaStream_t s = as_stream(stream);
-  cudaError_t e = launch_w4a4_pack_codes(ex->gate_up_q, ex->E, 0, gu_pk, s);
-  if (e == cudaSuccess) e = launch_w4a4_pack_codes(ex->down_q, ex->E, 1, dn_pk, s);
-  if (e == cudaSuccess) e = launch_w4a4_pack_scales(ex->gate_up_s, ex->E, 0, gu_sf, s);
+  cudaError_t e = launch_pack_codes(ex->gate_up_q, ex->E, 0, gu_pk, s);
+  if (e == cudaSuccess) e = launch_pack_codes(ex->down_q, ex->E, 1, dn_pk, s);
+  return cuda_status(e);
+}
+
+nvfp4_status moe_w4a4_pack_scales(const moe_experts* ex, uint8_t* gu_sf, uint8_t* dn_sf, void* stream) {
+  nvfp4_status st = check_experts(ex);
+  if (st != NVFP4_OK) return st;
+  if (!gu_sf || !dn_sf) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(gu_sf, 16) || !aligned(dn_sf, 16)) return NVFP4_ERR_ALIGNMENT;
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = launch_w4a4_pack_scales(ex->gate_up_s, ex->E, 0, gu_sf, s);
   if (e == cudaSuccess) e = launch_w4a4_pack_scales(ex->down_s, ex->E, 1, dn_sf, s);
   return cuda_status(e);
 }
@@ -736,7 +749,7 @@ static nvfp4_status w4a4_forward_impl(const void* x, int32_t T, const moe_expert
                             L.nt, aq, asf, roww, status, s);
   if (e != cudaSuccess || !mark(2)) return cuda_fail(e);
   W4A4Args ga;
-  ga.wq = ex->gate_up_pk;
+  ga.wq = w.gate_up_pk;
   ga.wsf = ex->gate_up_sf;
   ga.wg = w.gate_up_g;
   ga.gin = ex->input_scale_gate_up;
@@ -752,7 +765,7 @@ static nvfp4_status w4a4_forward_impl(const void* x, int32_t T, const moe_expert
   ga.status = status;
   if ((e = launch_w4a4_gemm(ga, 0, L.nt, s)) != cudaSuccess || !mark(3)) return cuda_fail(e);
   W4A4Args da = ga;
-  da.wq = ex->down_pk;
+  da.wq = w.down_pk;
   da.wsf = ex->down_sf;
   da.wg = w.down_g;
   da.gin = ex->input_scale_down;

@@ -81,6 +81,9 @@ struct ExpertArgs {
   const uint8_t* dn_s;
   const float* dn_g;
   const uint16_t* dn_b;
+  // optional packed codes (moe_nvfp4_pack_codes); null: read gu_q / dn_q by TMA
+  const uint8_t* gu_pk;
+  const uint8_t* dn_pk;
   const uint16_t* x;        // bf16 [T, H] (the layer input)
   __half* xs;               // [S, H] activations in expert-sorted slot order
   const int* meta;
@@ -113,9 +116,10 @@ cudaError_t launch_moe_down(const ExpertArgs& a, int nt, cudaStream_t st);
 int w4a4_tile_tokens(int T);
 // Packed block scales / codes of one projection (kind 0 gate_up, 1 down) of E experts.
 cudaError_t launch_w4a4_pack_scales(const uint8_t* s, int E, int kind, uint8_t* out, cudaStream_t st);
-cudaError_t launch_w4a4_pack_codes(const uint8_t* q, int E, int kind, uint8_t* out, cudaStream_t st);
-// Bytes of the packed codes of one projection (kind 0 gate_up, 1 down) of E experts.
-size_t w4a4_packed_code_bytes(int E, int kind);
+// Codes of one projection in 128-row x 256-element tiles, 128-byte swizzled
+// (moe_nvfp4_pack_codes), and their size.
+cudaError_t launch_pack_codes(const uint8_t* q, int E, int kind, uint8_t* out, cudaStream_t st);
+size_t packed_code_bytes(int E, int kind);
 // Each token's x -> E2M1 codes aq (tile-major, 128-byte swizzled) and scale
 // chunks asf (static global gx) at the padded rows of its 8 slots, and each
 // slot's routing weight at its padded row of roww [max_tiles*nt].

@@ -20,10 +20,13 @@
 // 64 up rows.  K is streamed in stages of 256 (gate_up 11, down 3 -- the last
 // one only 192 wide; the rest reads as zero).  A stage holds, in shared
 // memory:
-//   codes  128 rows x 128 B, 128B-swizzled, by ONE TMA box (gate_up: a 3-D
-//          box over {K bytes, row, gate/up half}, so 64 gate rows and their
-//          64 up rows come together; down: 128 consecutive rows).  Few large
-//          boxes keep the copy engine at full rate; narrow boxes do not.
+//   codes  128 rows x 128 B, 128B-swizzled: with the packed codes of
+//          moe_nvfp4_pack_codes, one contiguous 16 KB bulk copy (whole DRAM
+//          pages; gate_up tiles interleave 16 gate rows with their 16 up rows
+//          four times); else ONE TMA box (gate_up: a 3-D box over {K bytes,
+//          row, gate/up half}, so 64 gate rows and their 64 up rows come
+//          together; down: 128 consecutive rows) gathering 128-byte row
+//          pieces.
 //   x      the unit's 8 or 16 token rows x 256 K in f16, by one 3-D TMA box
 //          over {64 elements, K block, row} of the activations in
 //          expert-sorted order (x gathered for gate_up, h for down), so each
@@ -408,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_local = end - begin;
   if (n_local <= 0) return;  // uniform over the CTA, nothing issued
 
+  const uint8_t* pk = KIND == kGateUp ? p.gu_pk : p.dn_pk;
   if (warp == kProdWarp) {
     // -------------------------------------------------------------- producer
     if (lane == 0) {
@@ -428,7 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             const bool small = U[m].nvalid <= 8;
             mbar_arrive_expect_tx(&sm.full[slot], kCodeBytes + (small ? kXBytes / 2 : kXBytes));
-            if (KIND == kGateUp)  // {K bytes, row in half, gate/up half of expert e}
+            if (pk != nullptr)    // the packed tile (expert, row block, K stage)
+              bulk_g2s(sm.code[slot], pk + ((size_t)(U[m].e * C::NJ + U[m].j) * C::KC + kc) * kCodeBytes, kCodeBytes,
+                       &sm.full[slot]);
+            else if (KIND == kGateUp)  // {K bytes, row in half, gate/up half of expert e}
               tma_load_3d(smem_u32(sm.code[slot]), &tm_code, kc * 128, U[m].j * 64, U[m].e * 2, &sm.full[slot]);
             else
               tma_load_2d(smem_u32(sm.code[slot]), &tm_code, kc * 128, U[m].e * kH + U[m].j * kURows,
@@ -452,12 +459,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // units 8wq..8wq+7 in rows 0..63, their up rows in 64..127)
     const int rowA = KIND == kGateUp ? 8 * wq + g : 16 * wq + g;
     const int rowB = KIND == kGateUp ? 64 + 8 * wq + g : 16 * wq + g + 8;
+    // their rows in the stage's code tile: a packed gate_up tile holds gate
+    // unit u in row 32 (u / 16) + u % 16 and its up row 16 rows further
+    int tA = rowA, tB = rowB;
+    if (KIND == kGateUp && pk != nullptr) {
+      tA = 32 * (wq >> 1) + 8 * (wq & 1) + g;
+      tB = tA + 16;
+    }
     Lane<CODEC> L;
-    // code chunk cc = 2q + s of rows rowA / rowB (128B swizzle: chunk ^ (row & 7) = chunk ^ g)
+    // code chunk cc = 2q + s of rows tA / tB (128B swizzle: chunk ^ (row & 7) = chunk ^ g)
 #pragma unroll
     for (int s2 = 0; s2 < 2; ++s2) {
-      L.cA[s2] = (uint32_t)(rowA * 128 + (((2 * q + s2) ^ g) << 4));
-      L.cB[s2] = (uint32_t)(rowB * 128 + (((2 * q + s2) ^ g) << 4));
+      L.cA[s2] = (uint32_t)(tA * 128 + (((2 * q + s2) ^ g) << 4));
+      L.cB[s2] = (uint32_t)(tB * 128 + (((2 * q + s2) ^ g) << 4));
       // activation chunk 4s2 + i of the 128-byte row (token g, K block q): the
       // 128B swizzle XORs the chunk with that row's index 4g + q (mod 8)
       const int k = (4 * (g & 1) + q) & 7;

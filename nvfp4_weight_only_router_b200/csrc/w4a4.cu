@@ -19,8 +19,8 @@
 // index XOR-ed with the row index: the 128-byte swizzle), so the weight
 // stream reads whole 16 KB blocks of HBM.  Each expert's tokens are padded to
 // whole tiles of NT rows:
-//   weight codes      [E][N/128][K/256][128 rows][128 B]   (moe_w4a4_pack)
-//   weight scales     [E][N/128][K/64][512]                (moe_w4a4_pack)
+//   weight codes      [E][N/128][K/256][128 rows][128 B]   (moe_nvfp4_pack_codes)
+//   weight scales     [E][N/128][K/64][512]                (moe_w4a4_pack_scales)
 //   activation codes  [tiles][K/256][NT rows][128 B]
 //   activation scales [tiles][K/64][512]
 // A 512-byte chunk holds the 4 scales of one K step for 128 rows, row
@@ -602,7 +602,7 @@ cudaError_t launch_fp4(const W4A4Args& a, cudaStream_t st) {
 
 }  // namespace
 
-size_t w4a4_packed_code_bytes(int E, int kind) {
+size_t packed_code_bytes(int E, int kind) {
   return (size_t)E * (kind == 0 ? F4Dims<0>::NJ * F4Dims<0>::KCH : F4Dims<1>::NJ * F4Dims<1>::KCH) * kF4Rows * 128;
 }
 
@@ -617,7 +617,7 @@ cudaError_t launch_w4a4_pack_scales(const uint8_t* s, int E, int kind, uint8_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_w4a4_pack_codes(const uint8_t* q, int E, int kind, uint8_t* out, cudaStream_t st) {
+cudaError_t launch_pack_codes(const uint8_t* q, int E, int kind, uint8_t* out, cudaStream_t st) {
   const int64_t pieces = (int64_t)E * (kind == 0 ? F4Dims<0>::NJ * F4Dims<0>::KCH : F4Dims<1>::NJ * F4Dims<1>::KCH) *
                          kF4Rows * 8;
   const int blocks = (int)std::min<int64_t>((pieces + 255) / 256, 148 * 16);

@@ -25,7 +25,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported(capi):
     names = header_functions()
-    assert len(names) == 30
+    assert len(names) == 31
     for n in names:
         assert hasattr(capi.lib, n), n
         assert n in capi.SIGNATURES, n
@@ -38,7 +38,7 @@ def test_only_declared_symbols_are_exported(capi):
 
 
 def test_abi_version_and_status_strings(capi):
-    assert capi.nvfp4_abi_version() == 2
+    assert capi.nvfp4_abi_version() == 3
     for code in range(9):
         assert capi.status_string(code)
     assert capi.status_string(0) == "ok"
@@ -219,18 +219,40 @@ def test_aff4_validation(capi):
     assert c.moe_aff4_forward(P, 1, ctypes.byref(a), ctypes.byref(r), P, P, 0, None) == c.NVFP4_ERR_WORKSPACE
 
 
-def _w4a4(c, gx=0.003, gh=0.0007, sf=4096):
-    return c.moe_experts_w4a4(_experts(c), sf, sf, sf, sf, gx, gh)
+def _w4a4(c, gx=0.003, gh=0.0007, sf=4096, pk=4096):
+    x = _experts(c)
+    x.gate_up_pk, x.down_pk = pk, pk
+    return c.moe_experts_w4a4(x, sf, sf, gx, gh)
+
+
+def test_packing_validation(capi):
+    c = capi
+    assert c.moe_pack_bytes(128, 0) == 128 * 11 * 11 * 128 * 128      # 128-row tiles x 256-element chunks
+    assert c.moe_pack_bytes(128, 1) == 128 * 22 * 3 * 128 * 128
+    assert c.moe_pack_bytes(128, 2) == 128 * 1408 * 176
+    assert c.moe_pack_bytes(128, 3) == 128 * 2816 * 44
+    assert c.moe_pack_bytes(0, 0) == 0 and c.moe_pack_bytes(128, 4) == 0
+    P = 4096
+    x = _experts(c, I=512)
+    assert c.moe_nvfp4_pack_codes(ctypes.byref(x), P, P, None) == c.NVFP4_ERR_UNSUPPORTED
+    assert c.moe_nvfp4_pack_codes(ctypes.byref(_experts(c)), None, P, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_nvfp4_pack_codes(ctypes.byref(_experts(c)), P, P + 4, None) == c.NVFP4_ERR_ALIGNMENT
+    assert c.moe_w4a4_pack_scales(ctypes.byref(_experts(c)), P, None, None) == c.NVFP4_ERR_INVALID_ARG
+    assert c.moe_w4a4_pack_scales(ctypes.byref(_experts(c)), P + 8, P, None) == c.NVFP4_ERR_ALIGNMENT
+    # the packed codes of a forward: both or neither, aligned
+    r = _router(c)
+    one = _experts(c)
+    one.gate_up_pk = P
+    n = c.moe_forward_workspace_bytes(1, ctypes.byref(_experts(c)), ctypes.byref(r))
+    assert c.moe_forward_workspace_bytes(1, ctypes.byref(one), ctypes.byref(r)) == 0
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(one), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_INVALID_ARG
+    one.down_pk = P + 4
+    assert c.moe_nvfp4_forward(P, 1, ctypes.byref(one), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_ALIGNMENT
 
 
 def test_w4a4_validation(capi):
     c = capi
     r, w = _router(c), _w4a4(c)
-    assert c.moe_w4a4_pack_bytes(128, 0) == 128 * 11 * 11 * 128 * 128      # 128-row tiles x 256-element chunks
-    assert c.moe_w4a4_pack_bytes(128, 1) == 128 * 22 * 3 * 128 * 128
-    assert c.moe_w4a4_pack_bytes(128, 2) == 128 * 1408 * 176
-    assert c.moe_w4a4_pack_bytes(128, 3) == 128 * 2816 * 44
-    assert c.moe_w4a4_pack_bytes(0, 0) == 0 and c.moe_w4a4_pack_bytes(128, 4) == 0
     sizes = [c.moe_w4a4_workspace_bytes(T, ctypes.byref(w), ctypes.byref(r)) for T in (1, 64, 4096)]
     assert 0 < sizes[0] < sizes[1] < sizes[2]
     assert c.moe_w4a4_workspace_bytes(65537, ctypes.byref(w), ctypes.byref(r)) == 0
@@ -242,11 +264,8 @@ def test_w4a4_validation(capi):
     P, n = 4096, sizes[0]
     assert c.moe_w4a4_forward(P, 1, ctypes.byref(w), ctypes.byref(r), P, P, n - 1, None) == c.NVFP4_ERR_WORKSPACE
     assert c.moe_w4a4_forward(None, 1, ctypes.byref(w), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_INVALID_ARG
-    for bad in (_w4a4(c, gx=0.0), _w4a4(c, gh=float("inf")), _w4a4(c, gx=float("nan")), _w4a4(c, sf=None)):
+    for bad in (_w4a4(c, gx=0.0), _w4a4(c, gh=float("inf")), _w4a4(c, gx=float("nan")), _w4a4(c, sf=None),
+                _w4a4(c, pk=None)):
         assert c.moe_w4a4_forward(P, 1, ctypes.byref(bad), ctypes.byref(r), P, P, n, None) == c.NVFP4_ERR_INVALID_ARG
     assert c.moe_w4a4_forward(P, 1, ctypes.byref(_w4a4(c, sf=4096 + 8)), ctypes.byref(r), P, P, n,
                               None) == c.NVFP4_ERR_ALIGNMENT
-    x = _experts(c, I=512)
-    assert c.moe_w4a4_pack(ctypes.byref(x), P, P, P, P, None) == c.NVFP4_ERR_UNSUPPORTED
-    assert c.moe_w4a4_pack(ctypes.byref(_experts(c)), None, P, P, P, None) == c.NVFP4_ERR_INVALID_ARG
-    assert c.moe_w4a4_pack(ctypes.byref(_experts(c)), P, P, P + 4, P, None) == c.NVFP4_ERR_ALIGNMENT

@@ -78,6 +78,31 @@ def test_forward_decode_shapes(layer0, dev, T):
     check_forward(bf16_from_dev(y), y64)
 
 
+@pytest.fixture(scope="module")
+def packed_experts(layer0):
+    return layer0["dex"].packed()
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 256, 300])
+def test_forward_packed_codes(layer0, packed_experts, dev, T):
+    """With the packed code tiles the decode GEMVs (T <= 256) stream whole
+    16 KB blocks; the arithmetic is unchanged, so y is bit-identical to the
+    forward on the plain codes (T = 300 takes the tensor-core GEMMs, which read
+    the plain codes either way); on few tokens also against the oracle."""
+    ex, rt = layer0["ex"], layer0["rt"]
+    plain = lib.MoeLayer(layer0["dex"], layer0["drt"], max_tokens=T)
+    packed = lib.MoeLayer(packed_experts, layer0["drt"], max_tokens=T)
+    x = gen.make_x(1100 + T, T)
+    y1 = _run(plain, x, dev)
+    y2 = _run(packed, x, dev)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    if T <= 8:
+        ids = packed.views(T)["ids"].cpu().numpy()
+        ids0, _, logits = M.route(x, rt)
+        differ = check_ids(ids, ids0, logits)
+        check_forward(bf16_from_dev(y2), _oracle_y(x, ex, rt, ids, differ))
+
+
 def test_forward_repeat_is_deterministic(layer0, dev):
     layer = lib.MoeLayer(layer0["dex"], layer0["drt"], max_tokens=64)
     xd = bf16_to_dev(gen.make_x(77, 64), dev)

@@ -76,8 +76,8 @@ def test_pack_layout(layer, layer0):
     ex = layer0["ex"]
     Lq = np.arange(128)
     qd, w = Lq >> 5, Lq & 31
-    gu_pk = layer.gate_up_pk.cpu().numpy().reshape(E, 11, 11 * 128 * 128)
-    dn_pk = layer.down_pk.cpu().numpy().reshape(E, 22, 3 * 128 * 128)
+    gu_pk = layer.experts.gate_up_pk.cpu().numpy().reshape(E, 11, 11 * 128 * 128)
+    dn_pk = layer.experts.down_pk.cpu().numpy().reshape(E, 22, 3 * 128 * 128)
     gu = layer.gate_up_sf.cpu().numpy().reshape(E, 11, 44, 32, 4, 4)   # e, j, q, r0, r1, i
     dn = layer.down_sf.cpu().numpy().reshape(E, 22, 11, 32, 4, 4)
     L = np.arange(128).reshape(4, 32).T           # [r0, r1] -> tile row
