@@ -31,7 +31,9 @@
 // Tiles and warps as in the W4A16 tensor-core kernel: work tile = (expert,
 // token tile, 128 weight rows), K in 128-byte chunks (4 MMA K steps); warp 0
 // issues the bulk copies, warp 2 the copies of the block scales into tensor
-// memory, warp 1 the MMAs (one elected lane), warps 4-7 the epilogue.  A gate_up tile holds 64 hidden
+// memory, warp 1 the MMAs (one elected lane), warps 4.. the epilogue (one,
+// two or four sets of 4 warps for 16-, 64- and 128-token tiles, each set
+// taking a share of the tile's tokens).  A gate_up tile holds 64 hidden
 // units: lane quarter q has gate rows of units 16q.. in lanes 0-15 and the
 // matching up rows in lanes 16-31.  Every wait is bounded.
 #include <algorithm>
@@ -68,11 +70,11 @@ struct F4Cfg {
   static constexpr int STAGE = A_BYTES + B_BYTES + 2 * SF_BYTES;
   // epilogue: NEPI sets of 4 warps (one per tensor-memory lane quarter), set
   // h taking token columns [h TPS, (h + 1) TPS) of each tile
-  static constexpr int NEPI = NT >= 64 ? 2 : 1;
+  static constexpr int NEPI = NT >= 128 ? 4 : (NT >= 64 ? 2 : 1);
   static constexpr int TPS = NT / NEPI;
   static constexpr int THREADS = 32 * (kF4Epi0 + 4 * NEPI);
   static constexpr int STG = KIND == 0 ? TPS * 16 : 1;         // epilogue staging floats per warp
-  static constexpr int NS_SMEM = (224 * 1024 - 4 * 4 * STG) / STAGE;
+  static constexpr int NS_SMEM = (224 * 1024 - 4 * NEPI * 4 * STG) / STAGE;
   static constexpr int NS_TMEM = (kF4TmemCols - 2 * NT) / 32;  // 32 scale columns per stage
   static constexpr int NS_MIN = NS_SMEM < NS_TMEM ? NS_SMEM : NS_TMEM;
   static constexpr int NS = NS_MIN < 8 ? NS_MIN : 8;
