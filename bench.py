@@ -664,6 +664,14 @@ def run_ours(args, rank, world, local_rank):
         line["prefill"] = {k: p[k] for k in ("value", "unit", "ms_per_step", "roofline", "clocks", "e2e",
                                              "gpu_launches", "phase_ms_mean", "layer_tflops")}
         line["prefill"]["config"] = p["config"]
+    if args.workload == "decode64" and not args.no_w4a4:
+        # the W4A4 form of the same layer (NVFP4 activations on the FP4 tensor
+        # cores), decode and prefill, in the same invocation
+        for key, w in (("w4a4_decode", "w4a4_64"), ("w4a4_prefill", "w4a4_4096")):
+            q = measure(ctx, w, args, cpu_baseline=False)
+            line[key] = {k: q[k] for k in ("value", "unit", "ms_per_step", "roofline", "clocks", "e2e",
+                                           "gpu_launches", "phase_ms_mean", "dtype")}
+            line[key]["config"] = q["config"]
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -676,6 +684,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode64", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-w4a4", action="store_true",
+                    help="decode64: skip the W4A4 decode and prefill lines")
     ap.add_argument("--no-prefill", action="store_true",
                     help="decode64 only: skip the prefill4096 half of the metric")
     ap.add_argument("--min-warmup-s", type=float, default=1.0,
