@@ -264,18 +264,20 @@ __device__ __forceinline__ int padded_row(const int* prefix, const int* meta, in
   return prefix[lo] * nt + (pos - meta[kMetaOffsets + lo]);
 }
 
-// Each token's x quantised once under the static global gx (one warp per
-// token, one 16-element block per lane and step), its codes and scales
-// written to the padded rows of its 8 slots, and each slot's routing weight
-// to its padded row.  Padding rows are left as they are: a padding row only
-// feeds its own (unused) accumulator column.
+// Each token's x quantised once under the static global gx, its codes and
+// scales written to the padded rows of its 8 slots, and each slot's routing
+// weight to its padded row.  Work item = (token, 32 consecutive 16-element
+// blocks), one warp each, one block per lane, so that few tokens still spread
+// over many SMs.  Padding rows are left as they are: a padding row only feeds
+// its own (unused) accumulator column.
 template <int NT>
 __global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restrict__ x, const int* __restrict__ meta,
                                                         const int* __restrict__ slot_pos, int T, float gx,
                                                         const float* __restrict__ wts, uint8_t* __restrict__ aq,
                                                         uint8_t* __restrict__ asf, float* __restrict__ roww,
                                                         int* status) {
-  constexpr int NB = kH / kBlock;  // 176 blocks per row
+  constexpr int NB = kH / kBlock;          // 176 blocks per row
+  constexpr int NSEG = (NB + 31) / 32;     // 6 segments of 32 blocks (the last one 16)
   constexpr int KS = kH / 64;
   constexpr int KCH = kH / 256;
   __shared__ int prefix[kE + 1];
@@ -283,7 +285,8 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restri
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const TensorScale ts = scale_consts(gx);
-  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < T; t += gridDim.x * 8) {
+  for (int item = blockIdx.x * 8 + (threadIdx.x >> 5); item < T * NSEG; item += gridDim.x * 8) {
+    const int t = item / NSEG, seg = item % NSEG;
     // lanes 0..7: the padded row of slot j = lane (-1: a position outside the permutation)
     int R = 0;
     if (lane < kTopK) {
@@ -293,47 +296,45 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const uint16_t* __restri
         R = -1;
       } else {
         R = padded_row(prefix, meta, NT, pos);
-        roww[R] = wts[t * kTopK + lane];
+        if (seg == 0) roww[R] = wts[t * kTopK + lane];
       }
     }
     int rows[kTopK];
 #pragma unroll
     for (int j = 0; j < kTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, R, j);
-    for (int kb = lane; kb < NB + 16; kb += 32) {
-      // 192 lanes-steps: the last 16 lanes of the last step only gather scales
-      uint2 codes = make_uint2(0u, 0u);
-      uint32_t sc = 0;
-      if (kb < NB) {
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * kH + kb * kBlock);
-        const uint4 v0 = ldg_nc_v4(src), v1 = ldg_nc_v4(src + 1);
-        const uint32_t pr[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        float xv[16];
-        uint32_t key2 = 0;
+    const int kb = seg * 32 + lane;
+    uint2 codes = make_uint2(0u, 0u);
+    uint32_t sc = 0;
+    if (kb < NB) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * kH + kb * kBlock);
+      const uint4 v0 = ldg_nc_v4(src), v1 = ldg_nc_v4(src + 1);
+      const uint32_t pr[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      float xv[16];
+      uint32_t key2 = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          xv[2 * k] = bf16_bits_to_f32(pr[k] & 0xFFFFu);
-          xv[2 * k + 1] = bf16_bits_to_f32(pr[k] >> 16);
-          key2 = __vmaxu2(key2, pr[k] & 0x7FFF7FFFu);
-        }
-        sc = encode_block16f(xv, bf16_bits_to_f32(max(key2 & 0xFFFFu, key2 >> 16)), ts, codes);
+      for (int k = 0; k < 8; ++k) {
+        xv[2 * k] = bf16_bits_to_f32(pr[k] & 0xFFFFu);
+        xv[2 * k + 1] = bf16_bits_to_f32(pr[k] >> 16);
+        key2 = __vmaxu2(key2, pr[k] & 0x7FFF7FFFu);
       }
-      // the 4 scales of one MMA K step (lanes 4g..4g+3) as one word in lane 4g
-      uint32_t word = sc;
-      word |= __shfl_down_sync(0xffffffffu, sc, 1) << 8;
-      word |= __shfl_down_sync(0xffffffffu, sc, 2) << 16;
-      word |= __shfl_down_sync(0xffffffffu, sc, 3) << 24;
-      if (kb < NB) {
+      sc = encode_block16f(xv, bf16_bits_to_f32(max(key2 & 0xFFFFu, key2 >> 16)), ts, codes);
+    }
+    // the 4 scales of one MMA K step (lanes 4g..4g+3) as one word in lane 4g
+    uint32_t word = sc;
+    word |= __shfl_down_sync(0xffffffffu, sc, 1) << 8;
+    word |= __shfl_down_sync(0xffffffffu, sc, 2) << 16;
+    word |= __shfl_down_sync(0xffffffffu, sc, 3) << 24;
+    if (kb < NB) {
 #pragma unroll
-        for (int j = 0; j < kTopK; ++j) {
-          const int Rj = rows[j];
-          if (Rj < 0) continue;
-          const int tile = Rj / NT, r = Rj % NT;
-          const int c = kb >> 4, kbyte = (kb & 15) * 8;
-          *reinterpret_cast<uint2*>(aq + ((size_t)tile * KCH + c) * (NT * 128) + sw128(r, kbyte)) = codes;
-          if ((kb & 3) == 0)
-            *reinterpret_cast<uint32_t*>(asf + ((size_t)tile * KS + (kb >> 2)) * kSfChunk + 16 * (r & 31) + 4 * (r >> 5)) =
-                word;
-        }
+      for (int j = 0; j < kTopK; ++j) {
+        const int Rj = rows[j];
+        if (Rj < 0) continue;
+        const int tile = Rj / NT, r = Rj % NT;
+        const int c = kb >> 4, kbyte = (kb & 15) * 8;
+        *reinterpret_cast<uint2*>(aq + ((size_t)tile * KCH + c) * (NT * 128) + sw128(r, kbyte)) = codes;
+        if ((kb & 3) == 0)
+          *reinterpret_cast<uint32_t*>(asf + ((size_t)tile * KS + (kb >> 2)) * kSfChunk + 16 * (r & 31) + 4 * (r >> 5)) =
+              word;
       }
     }
   }
@@ -631,7 +632,7 @@ cudaError_t launch_pack_codes(const uint8_t* q, int E, int kind, uint8_t* out, c
 cudaError_t launch_w4a4_act_quant(const uint16_t* x, const int* meta, const int* slot_pos, const float* wts, int T,
                                   float gx, int nt, uint8_t* aq, uint8_t* asf, float* roww, int* status,
                                   cudaStream_t st) {
-  const int blocks = (int)std::min<int64_t>((T + 7) / 8, 148 * 8);
+  const int blocks = (int)std::min<int64_t>(((int64_t)T * 6 + 7) / 8, 148 * 8);  // 6 work items per token
   switch (nt) {
     case 16: act_quant_kernel<16><<<blocks, 256, 0, st>>>(x, meta, slot_pos, T, gx, wts, aq, asf, roww, status); break;
     case 64: act_quant_kernel<64><<<blocks, 256, 0, st>>>(x, meta, slot_pos, T, gx, wts, aq, asf, roww, status); break;
