@@ -94,7 +94,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 
 // ------------------------------------------------------------ tensor copies
-// TMA loads (no multicast) into this CTA's shared memory, completing on an
+// TMA loads into this CTA's own shared memory only, completing on an
 // mbarrier with a transaction count.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar) {
