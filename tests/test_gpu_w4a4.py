@@ -126,12 +126,25 @@ def _check_valid_rounding(codes, scales, h):
     assert np.all((v_lo <= v) & (v <= v_hi)), "hidden code outside its rounding range"
 
 
-@pytest.mark.parametrize("T", [1, 8, 64, 300, 2048])
-def test_w4a4_forward(layer, layer0, dev, T):
-    """T <= 256: 16-token tiles; 300: 64; 2048: 128 (the oracle on 12 sampled
-    tokens above 64)."""
+def _saturating_x(T, seed):
+    """x with some 16-element blocks scaled by 40 (|x| up to ~200): their block
+    scale saturates at 448 under Gx (whose range is 8) and their largest codes
+    at 6, the method's satfinite behaviour."""
+    x = F.bf16_to_f32(gen.make_x(seed, T)).copy()
+    rng = np.random.default_rng(seed)
+    for t in range(T):
+        for b in rng.choice(H // 16, 6, replace=False):
+            x[t, 16 * b:16 * b + 16] *= 40.0
+    return gen.bf16_bits(x)
+
+
+@pytest.mark.parametrize("T,kind", [(1, "n"), (8, "n"), (64, "n"), (256, "n"), (257, "n"), (300, "n"), (1025, "n"),
+                                    (2048, "n"), (16, "sat")])
+def test_w4a4_forward(layer, layer0, dev, T, kind):
+    """T <= 256: 16-token tiles; 257..1024: 64; above: 128 (the oracle on 12
+    sampled tokens above 64); "sat": blocks whose scale saturates."""
     ex, rt = layer0["ex"], layer0["rt"]
-    x = gen.make_x(900 + T, T)
+    x = gen.make_x(900 + T, T) if kind == "n" else _saturating_x(T, 990)
     y, v = _run(layer, dev, x)
     nt = v["tile_tokens"]
     rows_of_pos = _padded_rows(v["counts"].astype(np.int64), v["offsets"].astype(np.int64), nt)
