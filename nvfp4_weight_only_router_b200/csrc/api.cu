@@ -1,5 +1,7 @@
 // C ABI of the NVFP4 MoE library: argument validation, workspace layout and
 // launch sequencing on the caller's stream.  See include/nvfp4moe.h.
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <cmath>
 #include <mutex>
@@ -36,6 +38,16 @@ int* nvfp4moe::device_status_ptr() {
 namespace {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// A named range on the calling host thread for profilers (NVTX): kernels
+// launched inside it carry its name in an nsys or ncu timeline.  Without a
+// tool attached the calls do nothing.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
@@ -265,6 +277,7 @@ size_t nvfp4_quantize_workspace_bytes(int64_t E, int64_t N, int64_t K) {
 
 nvfp4_status nvfp4_quantize(const void* w, int64_t E, int64_t N, int64_t K, uint8_t* q, uint8_t* s,
                             float* g, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nv("nvfp4_quantize");
   nvfp4_status st = check_quant_dims(E, N, K);
   if (st != NVFP4_OK) return st;
   if (!w || !q || !s || !g) return NVFP4_ERR_INVALID_ARG;
@@ -295,6 +308,7 @@ size_t moe_route_workspace_bytes(int32_t T, const moe_router* r) {
 
 nvfp4_status moe_route(const void* x, int32_t T, const moe_router* r, int32_t* ids, float* w,
                        void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nv("moe_route");
   if (T < 1 || T > 65536 || !x || !ids || !w) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_router(r, false);
   if (st != NVFP4_OK) return st;
@@ -391,6 +405,7 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const ExpertPtrs& ex,
     return cudaEventRecord(e, s) == cudaSuccess;
   };
   if (!mark(0)) return cuda_fail(cudaGetLastError());
+  NvtxRange nv(dense ? "moe_forward_dense" : "moe_forward");
 
   cudaError_t e = cudaMemsetAsync(at<int>(ws, L.meta), 0, L.meta.bytes, s);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -404,7 +419,10 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const ExpertPtrs& ex,
     ra.sorted_slot = at<int>(ws, L.sorted);
     ra.slot_pos = at<int>(ws, L.pos);
   }
-  if ((e = launch_route(ra, s)) != cudaSuccess || !mark(1)) return cuda_fail(e);
+  {
+    NvtxRange r("route");
+    if ((e = launch_route(ra, s)) != cudaSuccess || !mark(1)) return cuda_fail(e);
+  }
 
   PermuteArgs pa;
   pa.ids = ids;
@@ -449,24 +467,32 @@ static nvfp4_status forward_impl(const void* x, int32_t T, const ExpertPtrs& ex,
   xa.status = status;
   xa.xs = at<__half>(ws, L.xs);
   // the activations follow their slots into expert order (f16 for the MMAs)
-  if ((e = launch_gather_sorted(xa, s)) != cudaSuccess) return cuda_fail(e);
-  if (!mark(2)) return cuda_fail(cudaGetLastError());
+  {
+    NvtxRange r("gather");
+    if ((e = launch_gather_sorted(xa, s)) != cudaSuccess) return cuda_fail(e);
+    if (!mark(2)) return cuda_fail(cudaGetLastError());
+  }
   if (T <= kStreamMaxTokens) {
     // few tokens per expert: the weight stream bounds the step (streaming
     // GEMV with register dequantisation)
+    NvtxRange r("experts (streaming GEMV)");
     e = launch_gate_up_stream(xa, s);
     if (e != cudaSuccess || !mark(3)) return cuda_fail(e);
     e = launch_down_stream(xa, s);
     if (e != cudaSuccess || !mark(4)) return cuda_fail(e);
   } else {
     // many tokens per expert: tensor-core grouped GEMMs on expert-sorted rows
+    NvtxRange r("experts (tensor-core GEMMs)");
     const int nt = T <= 512 ? 64 : 192;  // about the tokens an expert gets
     e = launch_moe_gate_up(xa, nt, s);
     if (e != cudaSuccess || !mark(3)) return cuda_fail(e);
     e = launch_moe_down(xa, nt, s);
     if (e != cudaSuccess || !mark(4)) return cuda_fail(e);
   }
-  if (finalize && ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5))) return cuda_fail(e);
+  if (finalize) {
+    NvtxRange r("combine");
+    if ((e = launch_finalize(xa, s)) != cudaSuccess || !mark(5)) return cuda_fail(e);
+  }
   return NVFP4_OK;
 }
 
@@ -525,6 +551,7 @@ size_t moe_block_workspace_bytes(int32_t T, const moe_block* b) {
 
 nvfp4_status moe_block_forward(const void* x, int32_t T, const moe_block* b, void* y, void* ws, size_t ws_bytes,
                                void* stream) {
+  NvtxRange nv("moe_block_forward");
   if (T < 1 || T > kBlockMaxTokens || !x || !y) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_block(b);
   if (st != NVFP4_OK) return st;
@@ -716,6 +743,7 @@ static nvfp4_status w4a4_forward_impl(const void* x, int32_t T, const moe_expert
     return cudaEventRecord(evt, s) == cudaSuccess;
   };
   if (!mark(0)) return cuda_fail(cudaGetLastError());
+  NvtxRange nv("moe_w4a4_forward");
   cudaError_t e = cudaMemsetAsync(at<int>(ws, L.meta), 0, L.meta.bytes, s);
   if (e != cudaSuccess) return cuda_fail(e);
   int32_t* ids = at<int32_t>(ws, L.ids);
