@@ -225,6 +225,9 @@ NVFP4MOE_API nvfp4_status moe_route(const void* x_dev, int32_t T, const moe_rout
  * maximum), saturates and records NVFP4_ERR_RANGE in the device status.
  * x must be finite.
  *   x_dev bf16 [T, H] (in), y_dev bf16 [T, H] (out)
+ * When experts->gate_up_pk / down_pk are set (moe_nvfp4_pack_codes), the
+ * decode kernels (T <= 256) read the codes from them; the result is the same
+ * bit for bit.  Both or neither must be set (NVFP4_ERR_INVALID_ARG).
  * Requires 1 <= T <= 65536, E == 128, H == 2816, I == 704, top_k == 8.
  * Workspace: moe_forward_workspace_bytes(T, experts, router) bytes.
  * ------------------------------------------------------------------------- */
